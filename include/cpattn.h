@@ -1,0 +1,186 @@
+/*
+ * cpattn.h -- C ABI of libcpattn.so: causal scaled-dot-product attention
+ * evaluated the ring way (context parallel / RingAttention) on one GPU.
+ *
+ * What is computed.  For every (batch b, head h) and query row i,
+ *     O_i = sum_{j in A_i} softmax_j(scale * q_i . k_j) v_j,
+ *     LSE_i = log sum_{j in A_i} exp(scale * q_i . k_j)      (natural log)
+ * with A_i = { j <= i } when causal, all j otherwise.  "Configuring
+ * RingAttention+FlashAttention for CP" (devpress.csdn.net), section 1: each
+ * rank's Q takes turns against the K/V blocks of every rank and the results
+ * are aggregated; section 3, note 2: the mask is exact, nothing leaks.
+ *
+ * How it is evaluated.  The sequence is split over cp_size virtual ranks.
+ *   causal:     2*cp_size chunks of c = S / (2*cp_size) rows; rank r owns
+ *               chunks r and 2*cp_size-1-r (the zigzag of the same page,
+ *               section 5, item 1);
+ *   non-causal: cp_size contiguous chunks of c = S / cp_size rows.
+ * At ring step t rank r attends to the K/V of rank (r - t) mod cp_size (same
+ * page, section 3 code).  A (q chunk a, kv chunk b) block is SKIP when a < b,
+ * DIAG (masked j <= i) when a == b, FULL otherwise.  Each step yields a partial
+ * (O, LSE) per row; partials are combined by the log-sum-exp merge
+ *     L = max(La,Lb) + log(exp(La-M) + exp(Lb-M)),  O = e^(La-L) Oa + e^(Lb-L) Ob.
+ * "Megatron-LM source analysis: Context Parallel" (mieleap.com), section 5:
+ * the per-step attention call of the double-buffered ring loop.
+ *
+ * Conventions for every entry point.
+ *   - Tensors are caller-owned DEVICE pointers, contiguous, layout [B][H][S][D]
+ *     (LSE and per-row vectors [B][H][S]).  The library keeps no pointer after
+ *     the call returns and allocates no device memory on any call.
+ *   - dtype is cpattn_dtype: CPATTN_BF16 (bf16 in/out, fp32 accumulate) or
+ *     CPATTN_FP32 (fp32 in/out, fp32 arithmetic throughout).
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; argument and shape errors are returned before
+ *     anything is enqueued.  In-kernel failures (a bounded wait that ran out)
+ *     are recorded on the device and reported by cpattn_sync_status().
+ *   - Preconditions (CPATTN_ERR_SHAPE otherwise): B, H >= 1; S >= 1;
+ *     cp_size >= 1; D is 64 or 128; causal: S % (2*cp_size) == 0, non-causal:
+ *     S % cp_size == 0, and the chunk length c is a multiple of 16.  bf16
+ *     problems with c % 128 == 0 run on the tcgen05 tensor-core kernels, the
+ *     rest on the CUDA-core kernels.
+ *   - Pointers must be 16-byte aligned (CPATTN_ERR_ALIGN); scale must be
+ *     finite and > 0 (CPATTN_ERR_ARG).
+ */
+#ifndef CPATTN_H
+#define CPATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CPATTN_OK = 0,
+    CPATTN_ERR_ARG = 1,       /* null pointer, bad scale, bad step, bad capacity */
+    CPATTN_ERR_SHAPE = 2,     /* sizes violate the preconditions above */
+    CPATTN_ERR_DTYPE = 3,     /* unknown dtype */
+    CPATTN_ERR_ALIGN = 4,     /* a pointer is not 16-byte aligned */
+    CPATTN_ERR_CUDA = 5,      /* a CUDA runtime call or launch failed */
+    CPATTN_ERR_TIMEOUT = 6,   /* a bounded in-kernel wait ran out (reported later) */
+    CPATTN_ERR_WORKSPACE = 7  /* workspace missing or smaller than required */
+} cpattn_status;
+
+typedef enum { CPATTN_BF16 = 0, CPATTN_FP32 = 1 } cpattn_dtype;
+
+/* Block kinds in a plan row. */
+enum { CPATTN_SKIP = 0, CPATTN_FULL = 1, CPATTN_DIAG = 2 };
+
+/* Number of int32 fields in one plan row. */
+#define CPATTN_PLAN_FIELDS 6
+
+/*
+ * cpattn_plan -- host only, no GPU needed.
+ * Writes the ring schedule: one row of CPATTN_PLAN_FIELDS int32 per
+ * (rank r, step t, q slot, kv slot) in lexicographic order, SKIP rows included:
+ *     (r, t, q_chunk a, kv_chunk b, src_rank, kind)
+ * with src_rank = (r - t) mod cp_size, a the q slot's chunk of rank r and b
+ * the kv slot's chunk of rank src_rank.  Rows: cp_size*cp_size*4 causal,
+ * cp_size*cp_size non-causal.  out: host buffer of capacity rows
+ * (capacity*CPATTN_PLAN_FIELDS int32).  *n_rows is always set to the number of
+ * rows needed; CPATTN_ERR_ARG if capacity is too small (nothing written) or a
+ * pointer is null, CPATTN_ERR_SHAPE if S is not a multiple of the chunk count.
+ * Sources: ring rule and zigzag as cited at the top of this file.
+ */
+int cpattn_plan(int S, int cp_size, int causal, int32_t* out, int capacity, int* n_rows);
+
+/*
+ * cpattn_fwd -- the whole ring forward in one launch: every virtual rank, every
+ * step, partials merged on chip by the online (log-sum-exp) rescale, SKIP
+ * blocks never computed.
+ *   q, k, v : [B][H][S][D] input dtype (read)
+ *   o       : [B][H][S][D] input dtype (written)
+ *   lse     : [B][H][S] fp32, natural-log LSE of scale*q.k (written)
+ */
+int cpattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int S, int D, int cp_size, int causal, float scale, int dtype, void* stream);
+
+/*
+ * cpattn_fwd_step -- ring step `step` (0 <= step < cp_size) for all virtual
+ * ranks at once: each row's partial against the K/V that its rank holds at
+ * that step (both kv chunks of the source rank, SKIP blocks omitted).
+ *   o_part  : [B][H][S][D] fp32, normalised partial output (written)
+ *   lse_part: [B][H][S] fp32, partial LSE; -inf (and o_part = 0) where every
+ *             block of the row is SKIP at this step (written)
+ */
+int cpattn_fwd_step(const void* q, const void* k, const void* v, float* o_part,
+                    float* lse_part, int B, int H, int S, int D, int cp_size, int causal,
+                    float scale, int step, int dtype, void* stream);
+
+/*
+ * cpattn_merge -- in place: (o_acc, lse_acc) <- merge((o_acc, lse_acc),
+ * (o_part, lse_part)) for `rows` rows of D fp32 values, by the log-sum-exp
+ * rule at the top of this file.  A side with LSE = -inf contributes nothing
+ * (both -inf: o_acc and lse_acc unchanged).  The merge the pages leave
+ * unwritten: their listing adds partial outputs, which is wrong; this is the
+ * exact combination.  rows >= 0, D in {64, 128}.
+ */
+int cpattn_merge(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
+                 long rows, int D, void* stream);
+
+/*
+ * cpattn_finalize -- o[rows][D] (dtype) <- o_acc[rows][D] (fp32), rounding to
+ * nearest-even for bf16.
+ */
+int cpattn_finalize(const float* o_acc, void* o, long rows, int D, int dtype, void* stream);
+
+/*
+ * cpattn_bwd_workspace_bytes -- bytes of device workspace cpattn_bwd needs for
+ * this shape (fp32 dQ accumulator and per-row delta).  0 on bad sizes.
+ */
+size_t cpattn_bwd_workspace_bytes(int B, int H, int S, int D);
+
+/*
+ * cpattn_bwd -- recompute backward from (O, LSE): for every non-SKIP block,
+ * P = exp(scale q.k - LSE) (DIAG masked), dV += P^T dO, dP = dO V^T,
+ * dS = P (dP - delta) with delta_i = dO_i . O_i, dK += scale dS^T Q,
+ * dQ += scale dS K.  The gradient is that of the same function the forward
+ * computes ("Megatron-LM source analysis: Context Parallel", section 2: the
+ * backward mirrors the forward's communication).
+ *   q, k, v, o, dout : [B][H][S][D] dtype (read); lse: [B][H][S] fp32 from
+ *                      cpattn_fwd (read)
+ *   dq, dk, dv       : [B][H][S][D] dtype (written)
+ *   workspace        : caller-owned device buffer of ws_bytes >=
+ *                      cpattn_bwd_workspace_bytes(B, H, S, D), 256-byte aligned;
+ *                      contents on entry are ignored
+ */
+int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+               int cp_size, int causal, float scale, void* workspace, size_t ws_bytes,
+               int dtype, void* stream);
+
+/*
+ * cpattn_sync_status -- synchronises `stream`, then returns and clears the
+ * device-side error word of the current device (CPATTN_OK, CPATTN_ERR_TIMEOUT)
+ * or CPATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+int cpattn_sync_status(void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* cpattn_status_str(int status);
+
+/*
+ * Diagnostics.
+ * cpattn_launch_count: number of kernels this library has enqueued so far in
+ *   this process (all devices).
+ * cpattn_set_path: 0 = automatic (tcgen05 kernels where the shape allows),
+ *   1 = force the CUDA-core kernels.  Returns the previous setting.  For tests
+ *   that compare the two kernel families.
+ * cpattn_last_path: kernel family used by the last fwd/bwd call
+ *   (0 tcgen05, 1 CUDA cores).
+ * cpattn_debug_stall: n > 0 makes the next n tcgen05 forward launches omit one
+ *   K/V tile load, so the bounded waits run out and the call reports
+ *   CPATTN_ERR_TIMEOUT through cpattn_sync_status; the device stays usable.
+ *   For failure-detection tests only.
+ */
+long long cpattn_launch_count(void);
+int cpattn_set_path(int path);
+int cpattn_last_path(void);
+int cpattn_debug_stall(int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CPATTN_H */

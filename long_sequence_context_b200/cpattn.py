@@ -1,0 +1,204 @@
+"""Python binding of libcpattn.so (the C ABI declared in include/cpattn.h).
+
+Argument marshalling only: every function checks device / dtype / contiguity,
+passes raw device pointers and the current CUDA stream to the library, and
+turns a non-zero status into an exception.  All arithmetic runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback.  If the shared
+library has not been built, importing this module raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcpattn.so")
+
+OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(8)
+BF16, FP32 = 0, 1
+SKIP, FULL, DIAG = 0, 1, 2
+PLAN_FIELDS = 6
+
+# every symbol include/cpattn.h declares
+EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpattn_finalize",
+           "cpattn_bwd_workspace_bytes", "cpattn_bwd", "cpattn_sync_status",
+           "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
+           "cpattn_debug_stall"]
+
+
+class CpattnError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m long_sequence_context_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, l, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_long, ctypes.c_size_t
+    sigs = {
+        "cpattn_plan": ([i, i, i, vp, i, ctypes.POINTER(ctypes.c_int)], i),
+        "cpattn_fwd": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp], i),
+        "cpattn_fwd_step": ([vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp], i),
+        "cpattn_merge": ([vp, vp, vp, vp, l, i, vp], i),
+        "cpattn_finalize": ([vp, vp, l, i, i, vp], i),
+        "cpattn_bwd_workspace_bytes": ([i, i, i, i], sz),
+        "cpattn_bwd": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, i, vp], i),
+        "cpattn_sync_status": ([vp], i),
+        "cpattn_status_str": ([i], ctypes.c_char_p),
+        "cpattn_launch_count": ([], ctypes.c_longlong),
+        "cpattn_set_path": ([i], i),
+        "cpattn_last_path": ([], i),
+        "cpattn_debug_stall": ([i], i),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.cpattn_status_str(int(status)).decode()
+
+
+def _check(status, where):
+    if status != OK:
+        raise CpattnError(status, where)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def plan(S: int, cp_size: int, causal: bool):
+    """Ring schedule rows (r, t, q_chunk, kv_chunk, src_rank, kind); host only."""
+    n = ctypes.c_int(0)
+    st = lib.cpattn_plan(S, cp_size, int(causal), None, 0, ctypes.byref(n))
+    if st not in (OK, ERR_ARG) or n.value == 0:
+        _check(st if st != OK else ERR_SHAPE, "cpattn_plan")
+    buf = (ctypes.c_int32 * (n.value * PLAN_FIELDS))()
+    _check(lib.cpattn_plan(S, cp_size, int(causal), buf, n.value, ctypes.byref(n)), "cpattn_plan")
+    flat = list(buf)
+    return [tuple(flat[r * PLAN_FIELDS:(r + 1) * PLAN_FIELDS]) for r in range(n.value)]
+
+
+def fwd(q, k, v, cp_size: int, causal: bool = True, scale=None, out=None, lse=None, stream=None):
+    """Ring forward: returns (o, lse) with o like q and lse fp32 [B, H, S]."""
+    B, H, S, D = q.shape
+    scale = float(scale if scale is not None else D ** -0.5)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{n} must match q in shape and dtype")
+    st = lib.cpattn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse_t, "lse"),
+                        B, H, S, D, cp_size, int(causal), scale, _dtype_code(q), _stream(stream))
+    _check(st, "cpattn_fwd")
+    return o, lse_t
+
+
+def fwd_step(q, k, v, cp_size: int, step: int, causal: bool = True, scale=None, stream=None):
+    """One ring step for every virtual rank: fp32 partial (o_part, lse_part)."""
+    B, H, S, D = q.shape
+    scale = float(scale if scale is not None else D ** -0.5)
+    o = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    st = lib.cpattn_fwd_step(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o_part"),
+                             _dev(lse, "lse_part"), B, H, S, D, cp_size, int(causal), scale, step,
+                             _dtype_code(q), _stream(stream))
+    _check(st, "cpattn_fwd_step")
+    return o, lse
+
+
+def merge_(o_acc, lse_acc, o_part, lse_part, stream=None):
+    """In-place log-sum-exp merge of (o_part, lse_part) into (o_acc, lse_acc)."""
+    D = o_acc.shape[-1]
+    rows = lse_acc.numel()
+    for t in (o_acc, lse_acc, o_part, lse_part):
+        if t.dtype != torch.float32:
+            raise TypeError("merge operands are fp32")
+    st = lib.cpattn_merge(_dev(o_acc, "o_acc"), _dev(lse_acc, "lse_acc"), _dev(o_part, "o_part"),
+                          _dev(lse_part, "lse_part"), rows, D, _stream(stream))
+    _check(st, "cpattn_merge")
+    return o_acc, lse_acc
+
+
+def finalize(o_acc, dtype=torch.bfloat16, stream=None):
+    D = o_acc.shape[-1]
+    o = torch.empty(o_acc.shape, dtype=dtype, device=o_acc.device)
+    st = lib.cpattn_finalize(_dev(o_acc, "o_acc"), _dev(o, "o"), o_acc.numel() // D, D,
+                             _dtype_code(o), _stream(stream))
+    _check(st, "cpattn_finalize")
+    return o
+
+
+def bwd_workspace_bytes(B, H, S, D) -> int:
+    return int(lib.cpattn_bwd_workspace_bytes(B, H, S, D))
+
+
+def bwd(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=None, workspace=None,
+        dq=None, dk=None, dv=None, stream=None):
+    """Recompute backward: returns (dq, dk, dv) like q."""
+    B, H, S, D = q.shape
+    scale = float(scale if scale is not None else D ** -0.5)
+    need = bwd_workspace_bytes(B, H, S, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    st = lib.cpattn_bwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"),
+                        _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),
+                        B, H, S, D, cp_size, int(causal), scale,
+                        ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
+                        _dtype_code(q), _stream(stream))
+    _check(st, "cpattn_bwd")
+    return dq, dk, dv
+
+
+def sync_status(stream=None) -> int:
+    return int(lib.cpattn_sync_status(_stream(stream)))
+
+
+def check_device_status(stream=None):
+    _check(sync_status(stream), "device status")
+
+
+def launch_count() -> int:
+    return int(lib.cpattn_launch_count())
+
+
+def set_path(path: int) -> int:
+    return int(lib.cpattn_set_path(int(path)))
+
+
+def last_path() -> int:
+    return int(lib.cpattn_last_path())
+
+
+def debug_stall(n: int) -> int:
+    return int(lib.cpattn_debug_stall(int(n)))

@@ -1,0 +1,53 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernel translation units.  Every launcher enqueues on `stream`, returns the
+// number of kernels it enqueued (>= 0) or -1 when a launch failed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ring.cuh"
+
+namespace cpattn {
+
+struct AttnShape {
+  int B, H, S, D;
+  RingGeom g;
+  float scale;
+  int bf16;  // 1: bf16 tensors, 0: fp32 tensors
+};
+
+// ---- CUDA-core kernels (any dtype, D in {64,128}, chunk % 16 == 0) ----
+// steps [t0, t1) of the ring; final=1 writes O in the input dtype, final=0
+// writes the fp32 normalised partial.  lse always fp32.
+int launch_simt_fwd(const AttnShape& sh, const void* q, const void* k, const void* v, void* o,
+                    float* lse, int t0, int t1, int final_out, unsigned* err,
+                    cudaStream_t stream);
+int launch_merge(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
+                 long rows, int D, cudaStream_t stream);
+int launch_finalize(const float* o_acc, void* o, long rows, int D, int bf16,
+                    cudaStream_t stream);
+// backward: delta = rowsum(dO * O) into ws_delta, then dK/dV (key-owned) and
+// dQ (row-owned) kernels; no atomics.
+int launch_simt_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
+                    const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                    void* dv, float* ws_delta, cudaStream_t stream);
+
+// ---- tcgen05 tensor-core kernels (bf16, D in {64,128}, chunk % 128 == 0) ----
+int launch_tc_fwd(const AttnShape& sh, const void* q, const void* k, const void* v, void* o,
+                  float* lse, unsigned* err, int stall, cudaStream_t stream);
+// one ring step, fp32 normalised partial O and partial LSE (-inf where empty)
+int launch_tc_fwd_step(const AttnShape& sh, const void* q, const void* k, const void* v,
+                       float* o_part, float* lse_part, int step, unsigned* err,
+                       cudaStream_t stream);
+// workspace layout: [dq_acc fp32 B*H*S*D][delta fp32 B*H*S]
+int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
+                  const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                  void* dv, float* ws_dq, float* ws_delta, unsigned* err, cudaStream_t stream);
+bool tc_fwd_supported(const AttnShape& sh);
+bool tc_bwd_supported(const AttnShape& sh);
+
+int num_sms(int device);
+
+}  // namespace cpattn
