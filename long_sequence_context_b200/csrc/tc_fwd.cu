@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(384, 1)
       int j = 0, tile, dg;
       bool ok = true;
       while (kv.next(P, tile, dg)) {
-        if (!mbar_wait(&s_ready[wg], s_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_ready[wg], s_cnt & 1, abort_flag, P.err)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
         uint32_t r[128];
@@ -248,15 +248,15 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
         const float m_tile = mx * P.sl2;
-        if (m_tile > m + kRescaleThreshold || m == -INFINITY) {
-          const float m_new = fmaxf(m, m_tile);
-          if (m != -INFINITY && m_new > m) {
-            const float f = ex2(m - m_new);
-            l *= f;
-            if (j > 0) rescale_rows<D>(tO, f);
-          }
-          m = m_new;
-        }
+        float m_new = m;
+        if (m_tile > m + kRescaleThreshold || m == -INFINITY) m_new = fmaxf(m, m_tile);
+        const bool grow = (m != -INFINITY) && (m_new > m);
+        const float f = grow ? ex2(m - m_new) : 1.f;
+        l *= f;
+        // TMEM loads / stores are warp-collective: the whole warp rescales
+        // (factor 1 for rows whose maximum stayed) when any row needs it
+        if (j > 0 && __any_sync(0xffffffffu, grow)) rescale_rows<D>(tO, f);
+        m = m_new;
         const float base = (m == -INFINITY) ? 0.f : m;
         float lsum = 0.f;
 #pragma unroll
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         continue;
       }
-      if (!mbar_wait(&o_ready[wg], o_cnt & 1, abort_flag, P.err)) break;
+      if (!mbar_wait_warp(&o_ready[wg], o_cnt & 1, abort_flag, P.err)) break;
       ++o_cnt;
       tc_fence_after();
       const float inv = 1.f / l;
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(384, 1)
       int tile, dg;
       KvIter probe = kv;
       if (!probe.next(P, tile, dg)) continue;  // empty item: nothing to load
-      if (n_items > 0 && !mbar_wait(q_empty, (n_items - 1) & 1, abort_flag, P.err)) break;
+      if (n_items > 0 && !mbar_wait_warp(q_empty, (n_items - 1) & 1, abort_flag, P.err)) break;
       const int rowbase = it.bh * S;
       if (lane == 0) {
         mbar_expect_tx(q_full, 2 * C::kTileBytes);
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int which = 0; which < 2; ++which) {
           const int s = kv_idx % C::kStages;
           if (kv_idx >= (uint32_t)C::kStages &&
-              !mbar_wait(&kv_empty[s], ((kv_idx / C::kStages) - 1) & 1, abort_flag, P.err)) {
+              !mbar_wait_warp(&kv_empty[s], ((kv_idx / C::kStages) - 1) & 1, abort_flag, P.err)) {
             ok = false;
             break;
           }
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(384, 1)
       int tile, dg;
       KvIter probe = kv;
       if (!probe.next(P, tile, dg)) continue;
-      if (!mbar_wait(q_full, n_items & 1, abort_flag, P.err)) break;
+      if (!mbar_wait_warp(q_full, n_items & 1, abort_flag, P.err)) break;
       ++n_items;
       tc_fence_after();
       bool has_prev = false, prev_first = true;
@@ -419,10 +419,10 @@ __global__ void __launch_bounds__(384, 1)
         ++kv_idx;
         const uint32_t sV = kv_idx % C::kStages, phV = (kv_idx / C::kStages) & 1;
         ++kv_idx;
-        if (!mbar_wait(&kv_full[sK], phK, abort_flag, P.err)) { ok = false; break; }
+        if (!mbar_wait_warp(&kv_full[sK], phK, abort_flag, P.err)) { ok = false; break; }
         if (has_prev) {
-          if (!mbar_wait(&kv_full[prev_sV], prev_phV, abort_flag, P.err) ||
-              !mbar_wait(&p_ready[0], p_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+          if (!mbar_wait_warp(&kv_full[prev_sV], prev_phV, abort_flag, P.err) ||
+              !mbar_wait_warp(&p_ready[0], p_cnt & 1, abort_flag, P.err)) { ok = false; break; }
         }
         tc_fence_after();
         if (lane == 0) {
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         __syncwarp();
         if (has_prev) {
-          if (!mbar_wait(&p_ready[1], p_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_ready[1], p_cnt & 1, abort_flag, P.err)) { ok = false; break; }
           ++p_cnt;
           tc_fence_after();
         }
@@ -477,8 +477,8 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) tc_commit(q_empty);
       __syncwarp();
       // last tile's P.V for both Q tiles
-      if (!mbar_wait(&kv_full[prev_sV], prev_phV, abort_flag, P.err) ||
-          !mbar_wait(&p_ready[0], p_cnt & 1, abort_flag, P.err)) break;
+      if (!mbar_wait_warp(&kv_full[prev_sV], prev_phV, abort_flag, P.err) ||
+          !mbar_wait_warp(&p_ready[0], p_cnt & 1, abort_flag, P.err)) break;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t vb = aKV + prev_sV * C::kTileBytes;
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_commit(&o_ready[0]);
       }
       __syncwarp();
-      if (!mbar_wait(&p_ready[1], p_cnt & 1, abort_flag, P.err)) break;
+      if (!mbar_wait_warp(&p_ready[1], p_cnt & 1, abort_flag, P.err)) break;
       ++p_cnt;
       tc_fence_after();
       if (lane == 0) {
