@@ -1,0 +1,380 @@
+"""Benchmark: causal ring attention (zigzag context parallel) forward and
+forward+backward on B200, through the C ABI of libcpattn.so.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {cpattn,reference}]
+                    [--workload NAME]
+
+One step = the whole hot path over one batch: cpattn_fwd (every ring step,
+merged on chip) then cpattn_bwd (preprocess, recompute backward, dQ
+conversion).  Inputs are resident in HBM before the timed region; q, k, v, O,
+dO together are far larger than the 126 MB L2, so no flush is needed between
+steps.  Timing: CUDA events on the launch stream, barrier + synchronize on
+both sides, max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on the
+host cores over a bounded sample of the same workload, as a baseline arm.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "causal_b1h32s32768d128_cp8_bf16"
+METRIC = "causal ring-attn TFLOP/s fwd & fwd+bwd on 1 B200; % of BF16 tensor peak"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# --------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = str(gpu_index)
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", self.gpu, "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        med = statistics.median(sm) if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ dist setup --
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_sample(w, seconds_hint=10.0):
+    """fp64 oracle fwd+bwd over one head of the workload truncated to S' rows.
+
+    Returns (TFLOP/s, description, threads).  The algorithmic FLOPs of the sample
+    use the same counting as the GPU number (causal half, backward 2.5x)."""
+    import numpy as np
+    import torch
+    from long_sequence_context_b200.inputs import make_qkv
+    from oracle import oracle as orc
+    S_s = min(w.S, 4096)
+    q, k, v, do = make_qkv(1, 1, S_s, w.D, w.torch_dtype, seed=w.seed, qkv_scale=w.qkv_scale)
+    f = lambda t: t.float().numpy().astype(np.float64)
+    q, k, v, do = f(q), f(k), f(v), f(do)
+    dense = 4.0 * S_s * S_s * w.D
+    flops_one = (dense / 2 if w.causal else dense) * 3.5
+    total, reps, t0 = 0.0, 0, time.perf_counter()
+    while True:
+        orc.attn_fwd(q, k, v, w.causal, w.scale)
+        orc.attn_bwd(q, k, v, do, w.causal, w.scale)
+        reps += 1
+        total = time.perf_counter() - t0
+        if total >= seconds_hint or reps >= 50:
+            break
+    tfl = flops_one * reps / total / 1e12
+    desc = (f"fp64 oracle fwd+bwd, 1 head x S={S_s} (prefix length of the workload's shape, "
+            f"same D, dtype-rounded inputs), {reps} rep(s) in {total:.1f}s")
+    return tfl, desc, orc.threads()
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    from long_sequence_context_b200.inputs import make_qkv
+    from oracle import oracle as orc
+    S_s = min(w.S, 2048)
+    q, k, v, do = make_qkv(1, 1, S_s, w.D, w.torch_dtype, seed=w.seed, qkv_scale=w.qkv_scale)
+    f = lambda t: t.float().numpy().astype(np.float64)
+    q, k, v, do = f(q), f(k), f(v), f(do)
+    dense = 4.0 * S_s * S_s * w.D
+    flops_step = (dense / 2 if w.causal else dense) * 3.5
+
+    def step():
+        orc.attn_fwd(q, k, v, w.causal, w.scale)
+        orc.attn_bwd(q, k, v, do, w.causal, w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    val = flops_step * args.steps / dt / 1e12
+    sample = (f"fp64 oracle fwd+bwd per step over 1 head x S={S_s} of the workload's shape "
+              f"(dtype-rounded inputs)")
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                       "cp_size": w.cp_size, "causal": w.causal},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": orc.threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- GPU arm --
+def run_gpu(args, w):
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    from long_sequence_context_b200 import cpattn as cp
+    from long_sequence_context_b200.inputs import workload_inputs
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+
+    q, k, v, do = workload_inputs(w, with_dout=True)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    od = torch.empty_like(qd)
+    lsed = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    dqd, dkd, dvd = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    ws = torch.empty(cp.bwd_workspace_bytes(w.B, w.H, w.S, w.D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cp.fwd(qd, kd, vd, w.cp_size, w.causal, w.scale, out=od, lse=lsed)
+        if not args.fwd_only:
+            cp.bwd(qd, kd, vd, od, lsed, dod, w.cp_size, w.causal, w.scale, workspace=ws,
+                   dq=dqd, dk=dkd, dv=dvd)
+
+    for _ in range(args.warmup):
+        step()
+    st = cp.sync_status()
+    if st != cp.OK:
+        raise RuntimeError(f"warm-up failed: {cp.status_str(st)}")
+
+    # ---- timed region (device events, max over ranks) ----
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    n0 = cp.launch_count()
+    cp.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    cp.profile(False)
+    launches = cp.launch_count() - n0
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    clk = clocks.stop()
+    st = cp.sync_status()
+    if st != cp.OK:
+        raise RuntimeError(f"timed region failed: {cp.status_str(st)}")
+
+    ms_step = ms_total / args.steps
+    f_fwd, f_bwd = w.flops_fwd(), (0.0 if args.fwd_only else w.flops_bwd())
+    value = world * (f_fwd + f_bwd) * args.steps / (ms_total * 1e-3) / 1e12
+
+    per_kernel = {}
+    for kind, name in cp.KERNEL_KINDS.items():
+        ms, n = cp.profile_read(kind)
+        if n:
+            per_kernel[name] = {"ms_total": ms, "launches": n, "ms_avg": ms / n}
+    fwd_ms = per_kernel.get("tc_fwd", per_kernel.get("simt_fwd", {})).get("ms_avg")
+    fwd_tflops = f_fwd / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None
+
+    # dominant kernel and its roofline (tensor-bound: algorithmic FLOPs per launch)
+    alg_flops = {"tc_fwd": f_fwd, "simt_fwd": f_fwd, "tc_bwd": f_bwd,
+                 "simt_dkdv": 0.8 * f_bwd, "simt_dq": 0.2 * f_bwd}
+    dom = max(per_kernel, key=lambda n: per_kernel[n]["ms_total"])
+    peak = peaks["bf16_tflops_sustained"]
+    roof = None
+    if dom in alg_flops:
+        ach = alg_flops[dom] / (per_kernel[dom]["ms_avg"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
+                "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "unit": "TFLOP/s",
+                "frac": ach / peak, "frac_of_burst_peak": ach / peaks["bf16_tflops"],
+                "traffic": None}
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+        ho = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        hl = torch.empty((w.B, w.H, w.S), dtype=torch.float32).pin_memory()
+        hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
+
+        def e2e_step():
+            for h, d in ((hq, qd), (hk, kd), (hv, vd), (hdo, dod)):
+                d.copy_(h, non_blocking=True)
+            step()
+            for d, h in ((od, ho), (lsed, hl), (dqd, hdq), (dkd, hdk), (dvd, hdv)):
+                h.copy_(d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(2, min(args.steps, 5))
+        barrier(world)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
+        e2e = {"value": world * (f_fwd + f_bwd) * n_e2e / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": e2e_ms / n_e2e}
+
+    # ---- CPU baseline: the oracle on this host, rank 0, N == 1 only ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tfl, desc, threads = oracle_sample(w)
+        cpu = {"value": tfl, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                       "cp_size": w.cp_size, "causal": w.causal,
+                       "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs (q,k,v,O,dO ~1.3 GB) larger than L2; no flush"},
+            "fwd_tflops": fwd_tflops,
+            "fwd_frac_of_peak": (fwd_tflops / peaks["bf16_tflops"]) if fwd_tflops else None,
+            "fwd_bwd_frac_of_peak": value / world / peaks["bf16_tflops"],
+            "peaks": peaks,
+            "per_kernel_ms": per_kernel,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cpattn", choices=["cpattn", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-only", action="store_true", help="time the forward alone (profiling)")
+    ap.add_argument("--shape", default=None,
+                    help="B,H,S,D,cp_size,causal: a smaller case of the workload (profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from long_sequence_context_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.shape:
+        import dataclasses
+        B, H, S, D, N, c = (int(x) for x in args.shape.split(","))
+        w = dataclasses.replace(w, name=f"{w.name}@B{B}H{H}S{S}D{D}cp{N}c{c}", B=B, H=H, S=S, D=D,
+                                cp_size=N, causal=bool(c))
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -175,6 +175,19 @@ const char* cpattn_status_str(int status);
  *   For failure-detection tests only.
  */
 long long cpattn_launch_count(void);
+/*
+ * cpattn_profile: on != 0 starts per-kernel timing (a CUDA event pair recorded
+ *   on the launch stream around every kernel the library enqueues, up to 8192
+ *   kernels) and discards earlier records; 0 stops recording.  Returns the
+ *   previous setting.
+ * cpattn_profile_read: total milliseconds and launch count of one kernel kind
+ *   since the last cpattn_profile(1); waits for those events.  Kernel kinds:
+ *   0 tcgen05 forward, 1 CUDA-core forward, 2 merge, 3 finalize, 4 backward
+ *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 backward,
+ *   8 dQ conversion.
+ */
+int cpattn_profile(int on);
+int cpattn_profile_read(int kernel_kind, double* total_ms, long long* launches);
 int cpattn_set_path(int path);
 int cpattn_last_path(void);
 int cpattn_debug_stall(int n);

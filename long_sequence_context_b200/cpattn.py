@@ -23,7 +23,7 @@ PLAN_FIELDS = 6
 EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpattn_finalize",
            "cpattn_bwd_workspace_bytes", "cpattn_bwd", "cpattn_sync_status",
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
-           "cpattn_debug_stall"]
+           "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read"]
 
 
 class CpattnError(RuntimeError):
@@ -52,6 +52,8 @@ def _load():
         "cpattn_set_path": ([i], i),
         "cpattn_last_path": ([], i),
         "cpattn_debug_stall": ([i], i),
+        "cpattn_profile": ([i], i),
+        "cpattn_profile_read": ([i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], i),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(L, name)
@@ -202,3 +204,19 @@ def last_path() -> int:
 
 def debug_stall(n: int) -> int:
     return int(lib.cpattn_debug_stall(int(n)))
+
+
+KERNEL_KINDS = {0: "tc_fwd", 1: "simt_fwd", 2: "merge", 3: "finalize", 4: "bwd_delta",
+                5: "simt_dkdv", 6: "simt_dq", 7: "tc_bwd", 8: "dq_convert"}
+
+
+def profile(on: bool) -> int:
+    return int(lib.cpattn_profile(int(on)))
+
+
+def profile_read(kind: int):
+    """(total_ms, launches) of one kernel kind since profile(True)."""
+    ms = ctypes.c_double(0)
+    n = ctypes.c_longlong(0)
+    _check(lib.cpattn_profile_read(int(kind), ctypes.byref(ms), ctypes.byref(n)), "cpattn_profile_read")
+    return ms.value, n.value

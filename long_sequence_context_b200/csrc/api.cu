@@ -42,6 +42,20 @@ unsigned* err_word() {
   return g_err_ptr[dev];
 }
 
+// ---- optional per-kernel event timing ----
+struct ProfRec {
+  int id;
+  cudaEvent_t a, b;
+};
+constexpr int kProfPool = 8192;
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+cudaEvent_t g_prof_events[2 * kProfPool];
+int g_prof_created = 0;
+int g_prof_used = 0;
+ProfRec g_prof_recs[kProfPool];
+int g_prof_open_id = -1;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int count(int n) {
@@ -248,9 +262,56 @@ int cpattn_sync_status(void* stream) {
   return CPATTN_OK;
 }
 
+int cpattn_profile(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  const int prev = g_prof_on ? 1 : 0;
+  g_prof_on = on != 0;
+  if (g_prof_on) g_prof_used = 0;
+  return prev;
+}
+
+int cpattn_profile_read(int kernel_id, double* total_ms, long long* launches) {
+  if (!total_ms || !launches) return CPATTN_ERR_ARG;
+  *total_ms = 0.0;
+  *launches = 0;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (int i = 0; i < g_prof_used; ++i) {
+    if (g_prof_recs[i].id != kernel_id) continue;
+    if (cudaEventSynchronize(g_prof_recs[i].b) != cudaSuccess) return CPATTN_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, g_prof_recs[i].a, g_prof_recs[i].b) != cudaSuccess)
+      return CPATTN_ERR_CUDA;
+    *total_ms += ms;
+    *launches += 1;
+  }
+  return CPATTN_OK;
+}
+
 }  // extern "C"
 
 namespace cpattn {
+void prof_begin(int kernel_id, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on || g_prof_used >= kProfPool) return;
+  const int need = 2 * (g_prof_used + 1);
+  while (g_prof_created < need) {
+    if (cudaEventCreate(&g_prof_events[g_prof_created]) != cudaSuccess) return;
+    ++g_prof_created;
+  }
+  ProfRec& r = g_prof_recs[g_prof_used];
+  r.id = kernel_id;
+  r.a = g_prof_events[2 * g_prof_used];
+  r.b = g_prof_events[2 * g_prof_used + 1];
+  cudaEventRecord(r.a, stream);
+  g_prof_open_id = kernel_id;
+}
+void prof_end(int kernel_id, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on || g_prof_open_id != kernel_id || g_prof_used >= kProfPool) return;
+  cudaEventRecord(g_prof_recs[g_prof_used].b, stream);
+  ++g_prof_used;
+  g_prof_open_id = -1;
+}
 int num_sms(int device) {
   static int cache[kMaxDevices] = {0};
   if (device < 0 || device >= kMaxDevices) return 148;

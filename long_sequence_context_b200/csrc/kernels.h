@@ -50,4 +50,22 @@ bool tc_bwd_supported(const AttnShape& sh);
 
 int num_sms(int device);
 
+// Per-kernel timing for diagnostics: when enabled (cpattn_profile), every
+// launcher brackets each kernel with prof_begin / prof_end, which record a
+// pair of CUDA events on the launch stream.
+enum KernelId : int {
+  kKTcFwd = 0,
+  kKSimtFwd = 1,
+  kKMerge = 2,
+  kKFinalize = 3,
+  kKDelta = 4,
+  kKSimtDkdv = 5,
+  kKSimtDq = 6,
+  kKTcBwd = 7,
+  kKDqConvert = 8,
+  kKNumKernels = 9
+};
+void prof_begin(int kernel_id, cudaStream_t stream);
+void prof_end(int kernel_id, cudaStream_t stream);
+
 }  // namespace cpattn

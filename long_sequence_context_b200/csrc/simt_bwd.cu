@@ -220,14 +220,20 @@ int run_bwd(const AttnShape& sh, const void* q, const void* k, const void* v, co
   const T* V = static_cast<const T*>(v);
   const T* O = static_cast<const T*>(o);
   const T* dO = static_cast<const T*>(dout);
+  prof_begin(kKDelta, stream);
   delta_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(O, dO, ws_delta, rows);
+  prof_end(kKDelta, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
   dim3 grid(sh.S / kTile, sh.B * sh.H);
+  prof_begin(kKSimtDkdv, stream);
   dkdv_kernel<T, D><<<grid, 128, 0, stream>>>(Q, K, V, lse, dO, ws_delta, static_cast<T*>(dk),
                                               static_cast<T*>(dv), sh.g, sh.scale);
+  prof_end(kKSimtDkdv, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
+  prof_begin(kKSimtDq, stream);
   dq_kernel<T, D><<<grid, 128, 0, stream>>>(Q, K, V, lse, dO, ws_delta, static_cast<T*>(dq),
                                             sh.g, sh.scale);
+  prof_end(kKSimtDq, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
   return 3;
 }

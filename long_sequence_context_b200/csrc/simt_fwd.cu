@@ -216,6 +216,7 @@ int launch_simt_fwd(const AttnShape& sh, const void* q, const void* k, const voi
   (void)err;
   dim3 grid(sh.S / kRowsPerBlock, sh.B * sh.H);
   const float sl2 = sh.scale * kLog2e;
+  prof_begin(kKSimtFwd, stream);
   if (sh.bf16) {
     auto* qq = static_cast<const __nv_bfloat16*>(q);
     auto* kk = static_cast<const __nv_bfloat16*>(k);
@@ -233,6 +234,7 @@ int launch_simt_fwd(const AttnShape& sh, const void* q, const void* k, const voi
     else
       simt_fwd_kernel<float, 128><<<grid, 128, 0, stream>>>(qq, kk, vv, o, lse, sh.g, sl2, t0, t1, final_out);
   }
+  prof_end(kKSimtFwd, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
@@ -241,22 +243,26 @@ int launch_merge(float* o_acc, float* lse_acc, const float* o_part, const float*
   if (rows == 0) return 0;
   const int rpb = 256 / (D / 4);
   const long blocks = (rows + rpb - 1) / rpb;
+  prof_begin(kKMerge, stream);
   if (D == 64)
     merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(o_acc, lse_acc, o_part, lse_part, rows);
   else
     merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(o_acc, lse_acc, o_part, lse_part, rows);
+  prof_end(kKMerge, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
 int launch_finalize(const float* o_acc, void* o, long rows, int D, int bf16, cudaStream_t stream) {
   const long n4 = rows * D / 4;
   if (n4 == 0) return 0;
+  prof_begin(kKFinalize, stream);
   if (bf16)
     finalize_bf16_kernel<<<grid_for(n4, 256), 256, 0, stream>>>(
         reinterpret_cast<const float4*>(o_acc), reinterpret_cast<uint2*>(o), n4);
   else
     copy_f4_kernel<<<grid_for(n4, 256), 256, 0, stream>>>(reinterpret_cast<const float4*>(o_acc),
                                                           reinterpret_cast<float4*>(o), n4);
+  prof_end(kKFinalize, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 

@@ -553,7 +553,9 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   cudaGetDevice(&dev);
   int grid = num_sms(dev);
   if (grid > P.n_items) grid = P.n_items;
+  prof_begin(kKTcFwd, stream);
   tc_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, P);
+  prof_end(kKTcFwd, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
