@@ -150,6 +150,37 @@ int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const
                int cp_size, int causal, float scale, void* workspace, size_t ws_bytes,
                int dtype, void* stream);
 
+/* Size of the fixed device scratch array used by cpattn_bwd_noalloc (64 MiB). */
+#define CPATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * cpattn_bwd_noalloc -- the same backward as cpattn_bwd, for callers that
+ * cannot allocate device memory (code running inside an allocator's own
+ * callbacks, in a process whose memory pool belongs to another framework, or on
+ * a path that cannot afford an allocation's synchronisation or failure).  The
+ * pages have no counterpart: this is an interface convenience, not part of the
+ * method.
+ *   Arguments: as cpattn_bwd, minus the workspace.  The caller still passes
+ *   every input and output.
+ *   Scratch: a fixed CPATTN_NOALLOC_SCRATCH_BYTES array in device global
+ *   memory that every device loading this library holds until the process
+ *   exits.  The function itself allocates and frees nothing.
+ *   Limits: shapes whose cpattn_bwd_workspace_bytes(B, H, S, D) exceeds
+ *   CPATTN_NOALLOC_SCRATCH_BYTES are rejected with CPATTN_ERR_WORKSPACE before
+ *   anything is enqueued (CPATTN_ERR_SHAPE for invalid sizes).
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (with that device current); make that first call before any stream
+ *   capture begins.
+ *   Sharing: all calls on a device use the same array, which keeps the last
+ *   call's contents (the backward clears what it accumulates into).  Calls
+ *   that can overlap on the GPU -- on different streams, or from different
+ *   host threads -- race on the array; serialise them.
+ */
+int cpattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                       int H, int S, int D, int cp_size, int causal, float scale, int dtype,
+                       void* stream);
+
 /*
  * cpattn_sync_status -- synchronises `stream`, then returns and clears the
  * device-side error word of the current device (CPATTN_OK, CPATTN_ERR_TIMEOUT)

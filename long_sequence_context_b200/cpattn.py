@@ -23,7 +23,10 @@ PLAN_FIELDS = 6
 EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpattn_finalize",
            "cpattn_bwd_workspace_bytes", "cpattn_bwd", "cpattn_sync_status",
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
-           "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read"]
+           "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc"]
+
+# size of the library's fixed scratch array behind bwd_noalloc
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class CpattnError(RuntimeError):
@@ -52,6 +55,7 @@ def _load():
         "cpattn_set_path": ([i], i),
         "cpattn_last_path": ([], i),
         "cpattn_debug_stall": ([i], i),
+        "cpattn_bwd_noalloc": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp], i),
         "cpattn_profile": ([i], i),
         "cpattn_profile_read": ([i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], i),
     }
@@ -179,6 +183,25 @@ def bwd(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=None, wo
                         ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
                         _dtype_code(q), _stream(stream))
     _check(st, "cpattn_bwd")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=None,
+                dq=None, dk=None, dv=None, stream=None):
+    """Backward without a caller workspace: the library's fixed device scratch
+    array stands in for it (see cpattn_bwd_noalloc in include/cpattn.h).  For
+    callers that cannot allocate device memory, pass preallocated dq/dk/dv;
+    calls that may overlap on the GPU must be serialised by the caller."""
+    B, H, S, D = q.shape
+    scale = float(scale if scale is not None else D ** -0.5)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    st = lib.cpattn_bwd_noalloc(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"),
+                                _dev(lse, "lse"), _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"),
+                                _dev(dv, "dv"), B, H, S, D, cp_size, int(causal), scale,
+                                _dtype_code(q), _stream(stream))
+    _check(st, "cpattn_bwd_noalloc")
     return dq, dk, dv
 
 
