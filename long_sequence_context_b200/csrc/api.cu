@@ -9,7 +9,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "../../include/cpattn.h"
+#include "cpattn.h"
 #include "kernels.h"
 
 using namespace cpattn;

@@ -19,7 +19,7 @@
 
 #include <mutex>
 
-#include "../../include/cpattn.h"
+#include "cpattn.h"
 
 namespace {
 

@@ -57,8 +57,12 @@ struct BwdCfg {
   static constexpr int kOffQ = 2 * kTileBytes;  // stage s: Q at +2s*tile, dO at +(2s+1)*tile
   static constexpr int kOffDS = kOffQ + kQStages * 2 * kTileBytes;
   static constexpr int kDSBytes = 128 * 128 * 2;
-  static constexpr int kOffBar = kOffDS + kDSBytes;
-  static constexpr int kSmemBytes = 1024 + kOffBar + 256;
+  static constexpr int kOffLD = kOffDS + kDSBytes;  // stage s: LSE[128], delta[128] (fp32)
+  static constexpr int kLDBytes = 1024;
+  static constexpr int kOffBar = kOffLD + kQStages * kLDBytes;
+  // no alignment slack: the dynamic shared window starts 1024-byte aligned
+  // (checked at kernel entry)
+  static constexpr int kSmemBytes = kOffBar + 256;
   static constexpr bool kSplitDq = (D == 128);
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
   static constexpr uint32_t kColDK = (D == 128) ? 384 : 320;
@@ -75,6 +79,7 @@ struct BwdParams {
   int T;        // 128-row tiles per chunk
   int tiles;    // 128-row tiles per head (S / 128)
   int n_items;  // BH * tiles
+  int G;        // heads per scheduling group (divides BH)
   float sl2;    // scale * log2(e)
   float scale;
   const float* lse;
@@ -125,6 +130,16 @@ struct QIter {
   }
 };
 
+// Work index -> (K/V tile, head).  Heads are taken G at a time, so the CTAs
+// busy at any moment share a few heads' Q, dO and dQ accumulator in L2; inside
+// a group K/V tiles go in ascending position (most q tiles first).
+__device__ __forceinline__ void decode_item(const BwdParams& P, int w, int& jt, int& bh) {
+  const int per_group = P.G * P.tiles;
+  const int g = w / per_group, r = w % per_group;
+  jt = r / P.G;
+  bh = g * P.G + r % P.G;
+}
+
 __device__ __forceinline__ int snake_item(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
@@ -133,11 +148,14 @@ template <int D>
 __global__ void __launch_bounds__(320, 1)
     tc_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const BwdParams P) {
+                  const __grid_constant__ CUtensorMap tmdQ, const BwdParams P) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(P.err, kErrLayout);
+    return;
+  }
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sDS = smem + C::kOffDS;
@@ -153,7 +171,10 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* kv_done = bars + 10;
   uint64_t* acc_free = bars + 11;
   uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* stage_full = bars + 13;  // dQ rows written to the staging tile (128 arrivals)
+  uint64_t* stage_free = bars + 14;  // staging tile read by the TMA reduction
+  uint64_t* ds_free = bars + 15;     // dS buffer free again for the next q tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -171,6 +192,9 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(kv_done, 1);
     mbar_init(acc_free, 128);
     mbar_init(drain, 1);
+    mbar_init(stage_full, 128);
+    mbar_init(stage_free, 1);
+    mbar_init(ds_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -183,6 +207,7 @@ __global__ void __launch_bounds__(320, 1)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     prefetch_tensormap(&tmdO);
+    prefetch_tensormap(&tmdQ);
   }
   __syncthreads();
   tc_fence_after();
@@ -203,16 +228,27 @@ __global__ void __launch_bounds__(320, 1)
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
-      const int jt = w / P.BH, bh = w % P.BH;
+      int jt, bh;
+      decode_item(P, w, jt, bh);
       QIter qi;
       qi.init(P, jt);
       int qt, dg;
       while (qi.next(P, qt, dg)) {
         if (!mbar_wait_warp(s_ready, s_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+        // the dS buffer doubles as the dQ staging tile of the previous q tile
+        if (s_cnt > 0 && !mbar_wait_warp(ds_free, (s_cnt - 1) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+        // LSE and delta of this q tile arrived with its Q / dO stage
+        if (!mbar_wait_warp(&q_full[s_cnt & 1], (s_cnt >> 1) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+        const float4* lse4 = reinterpret_cast<const float4*>(smem + C::kOffLD + (s_cnt & 1) * C::kLDBytes);
+        const float4* dl4 = lse4 + 32;
         ++s_cnt;
         tc_fence_after();
-        const float4* lse4 = reinterpret_cast<const float4*>(P.lse + (long)bh * S + qt * 128);
-        const float4* dl4 = reinterpret_cast<const float4*>(P.delta + (long)bh * S + qt * 128);
 #pragma unroll
         for (int cb = 0; cb < 128; cb += 32) {
           uint32_t sv[32], dpv[32];
@@ -222,8 +258,8 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t pk[16], dsk[16];
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 L = __ldg(lse4 + (cb >> 2) + c4);
-            const float4 Dl = __ldg(dl4 + (cb >> 2) + c4);
+            const float4 L = lse4[(cb >> 2) + c4];
+            const float4 Dl = dl4[(cb >> 2) + c4];
             const float lv[4] = {L.x, L.y, L.z, L.w};
             const float dv_[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
             float p[4], ds[4];
@@ -293,12 +329,14 @@ __global__ void __launch_bounds__(320, 1)
     const int quarter = warp - 4;
     const int rloc = quarter * 32 + lane;  // query row within the q tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint32_t dq_cnt = 0;
+    const bool leader = (quarter == 0);  // warp 4 issues the TMA reductions
+    uint32_t dq_cnt = 0, use_cnt = 0, free_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
-      const int jt = w / P.BH, bh = w % P.BH;
+      int jt, bh;
+      decode_item(P, w, jt, bh);
       QIter qi;
       qi.init(P, jt);
       int qt, dg;
@@ -319,13 +357,45 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(dq_free);
-        float* dst = P.dq_acc + ((long)bh * S + (long)qt * 128 + rloc) * D;
+        // Add the tile into the fp32 accumulator with TMA reductions, 64
+        // columns at a time, staged in the dS buffer (free: the dQ MMA that
+        // read it is complete) as two 128-row x 32-column swizzled boxes.
 #pragma unroll
-        for (int c = 0; c < D; c += 4)
-          red_add_v4(dst + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                     __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+        for (int h = 0; h < D / 64; ++h) {
+          if (h > 0) {
+            if (!mbar_wait_warp(stage_free, free_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+            ++free_cnt;
+          }
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            uint8_t* rowp = sDS + b * C::kSubBytes + rloc * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int col = 64 * h + 32 * b + 4 * c;
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (rloc & 7)) << 4)) =
+                  make_uint4(v[col], v[col + 1], v[col + 2], v[col + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(stage_full);
+          if (leader) {
+            if (!mbar_wait_warp(stage_full, use_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+            if (lane == 0) {
+              const int y = bh * S + qt * 128;
+              tma_reduce_add_2d(&tmdQ, sDS, 64 * h, y);
+              tma_reduce_add_2d(&tmdQ, sDS + C::kSubBytes, 64 * h + 32, y);
+              bulk_commit_group();
+              bulk_wait_read_all();
+              mbar_arrive(h + 1 < D / 64 ? stage_free : ds_free);
+            }
+            __syncwarp();
+          }
+          ++use_cnt;
+        }
+        if (!ok) break;
       }
     }
+    if (leader && lane == 0) bulk_wait_all();
   } else if (warp == 8) {
     // ----------------------------------------------------------------- TMA --
     uint32_t items = 0, q_cnt = 0;
@@ -333,7 +403,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
-      const int jt = w / P.BH, bh = w % P.BH;
+      int jt, bh;
+      decode_item(P, w, jt, bh);
       const int rowbase = bh * S;
       if (items > 0 && !mbar_wait_warp(kv_empty, (items - 1) & 1, abort_flag, P.err)) break;
       if (lane == 0) {
@@ -358,12 +429,16 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) {
           uint8_t* sq = smem + C::kOffQ + (2 * st) * C::kTileBytes;
           uint8_t* sdo = sq + C::kTileBytes;
-          mbar_expect_tx(&q_full[st], 2 * C::kTileBytes);
+          uint8_t* sld = smem + C::kOffLD + st * C::kLDBytes;
+          mbar_expect_tx(&q_full[st], 2 * C::kTileBytes + C::kLDBytes);
 #pragma unroll
           for (int sb = 0; sb < D / 64; ++sb) {
             tma_load_2d(sq + sb * C::kSubBytes, &tmQ, &q_full[st], sb * 64, rowbase + qt * 128);
             tma_load_2d(sdo + sb * C::kSubBytes, &tmdO, &q_full[st], sb * 64, rowbase + qt * 128);
           }
+          const long r0 = (long)rowbase + qt * 128;
+          bulk_load(sld, P.lse + r0, 512, &q_full[st]);
+          bulk_load(sld + 512, P.delta + r0, 512, &q_full[st]);
         }
         __syncwarp();
         ++q_cnt;
@@ -389,7 +464,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
-      const int jt = w / P.BH;
+      int jt, bh;
+      decode_item(P, w, jt, bh);
       if (!mbar_wait_warp(kv_full, items & 1, abort_flag, P.err)) break;
       tc_fence_after();
       QIter qi;
@@ -533,9 +609,10 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
                 float* ws_delta, unsigned* err, cudaStream_t stream) {
   using C = BwdCfg<D>;
   const long rows = (long)sh.B * sh.H * sh.S;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_tmap_bf16_2d(&mq, q, rows, D, 64, 128) || !make_tmap_bf16_2d(&mk, k, rows, D, 64, 128) ||
-      !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128) || !make_tmap_bf16_2d(&mdo, dout, rows, D, 64, 128))
+      !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128) || !make_tmap_bf16_2d(&mdo, dout, rows, D, 64, 128) ||
+      !make_tmap_f32_2d(&mdq, ws_dq, rows, D, 32, 128))
     return -1;
   int launched = 0;
   prof_begin(kKDelta, stream);
@@ -552,6 +629,7 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.T = sh.g.c / 128;
   P.tiles = sh.S / 128;
   P.n_items = P.BH * P.tiles;
+  P.G = (P.BH % 2 == 0) ? 2 : 1;
   P.sl2 = sh.scale * kLog2e;
   P.scale = sh.scale;
   P.lse = lse;
@@ -572,7 +650,7 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   int grid = num_sms(dev);
   if (grid > P.n_items) grid = P.n_items;
   prof_begin(kKTcBwd, stream);
-  tc_bwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
+  tc_bwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, P);
   prof_end(kKTcBwd, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
   ++launched;

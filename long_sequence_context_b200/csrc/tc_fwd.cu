@@ -64,6 +64,7 @@ struct FwdParams {
   int T;           // 128-row tiles per chunk
   int pairs;       // work items per chunk: ceil(T / 2)
   int n_items;     // BH * n_chunks * pairs
+  int G;           // heads per scheduling group (divides BH)
   int t0, t1;      // ring steps [t0, t1)
   int out_f32;     // 1: fp32 normalised partial output, 0: bf16 output
   float sl2;       // scale * log2(e)
@@ -78,10 +79,13 @@ struct Item {
 };
 
 __device__ __forceinline__ void decode_item(const FwdParams& P, int w, Item& it) {
-  // descending global tile position = descending causal cost (LPT order);
-  // heads interleaved so neighbouring work indices cost the same
-  const int u = w / P.BH;
-  it.bh = w % P.BH;
+  // heads are taken G at a time (the CTAs busy at any moment share a few
+  // heads' K / V in L2); inside a group, descending global tile position =
+  // descending causal cost (longest first), heads interleaved
+  const int per_group = P.G * P.g.n_chunks * P.pairs;
+  const int grp = w / per_group, rem = w % per_group;
+  const int u = rem / P.G;
+  it.bh = grp * P.G + rem % P.G;
   const int a_rev = u / P.pairs, p_rev = u % P.pairs;
   it.a = P.g.n_chunks - 1 - a_rev;
   const int p = P.pairs - 1 - p_rev;
@@ -534,6 +538,7 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.T = sh.g.c / 128;
   P.pairs = (P.T + 1) / 2;
   P.n_items = P.BH * sh.g.n_chunks * P.pairs;
+  P.G = (P.BH % 4 == 0) ? 4 : (P.BH % 2 == 0) ? 2 : 1;
   P.t0 = t0;
   P.t1 = t1;
   P.out_f32 = out_f32;
