@@ -270,7 +270,9 @@ def run_gpu(args, w):
     fwd_tflops = f_fwd / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None
 
     # dominant kernel and its roofline (tensor-bound: algorithmic FLOPs per launch)
-    alg_flops = {"tc_fwd": f_fwd, "simt_fwd": f_fwd, "tc_bwd": f_bwd,
+    # backward split: the dK/dV kernels own S, dP, dV, dK (4 of the 5 matrix
+    # products), the dQ kernels own dQ (their S / dP recompute is not counted)
+    alg_flops = {"tc_fwd": f_fwd, "simt_fwd": f_fwd, "tc_dkdv": 0.8 * f_bwd, "tc_dq": 0.2 * f_bwd,
                  "simt_dkdv": 0.8 * f_bwd, "simt_dq": 0.2 * f_bwd}
     dom = max(per_kernel, key=lambda n: per_kernel[n]["ms_total"])
     peak = peaks["bf16_tflops_sustained"]

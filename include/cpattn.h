@@ -127,7 +127,8 @@ int cpattn_finalize(const float* o_acc, void* o, long rows, int D, int dtype, vo
 
 /*
  * cpattn_bwd_workspace_bytes -- bytes of device workspace cpattn_bwd needs for
- * this shape (fp32 dQ accumulator and per-row delta).  0 on bad sizes.
+ * this shape (two fp32 values per row: delta_i = dO_i . O_i and LSE_i in base
+ * 2).  0 on bad sizes.
  */
 size_t cpattn_bwd_workspace_bytes(int B, int H, int S, int D);
 
@@ -214,8 +215,8 @@ long long cpattn_launch_count(void);
  * cpattn_profile_read: total milliseconds and launch count of one kernel kind
  *   since the last cpattn_profile(1); waits for those events.  Kernel kinds:
  *   0 tcgen05 forward, 1 CUDA-core forward, 2 merge, 3 finalize, 4 backward
- *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 backward,
- *   8 dQ conversion.
+ *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 dK/dV,
+ *   8 tcgen05 dQ.
  */
 int cpattn_profile(int on);
 int cpattn_profile_read(int kernel_kind, double* total_ms, long long* launches);

@@ -230,7 +230,7 @@ def debug_stall(n: int) -> int:
 
 
 KERNEL_KINDS = {0: "tc_fwd", 1: "simt_fwd", 2: "merge", 3: "finalize", 4: "bwd_delta",
-                5: "simt_dkdv", 6: "simt_dq", 7: "tc_bwd", 8: "dq_convert"}
+                5: "simt_dkdv", 6: "simt_dq", 7: "tc_dkdv", 8: "tc_dq"}
 
 
 def profile(on: bool) -> int:

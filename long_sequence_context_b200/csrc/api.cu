@@ -211,10 +211,10 @@ int cpattn_finalize(const float* o_acc, void* o, long rows, int D, int dtype, vo
 
 size_t cpattn_bwd_workspace_bytes(int B, int H, int S, int D) {
   if (B < 1 || H < 1 || S < 1 || (D != 64 && D != 128)) return 0;
+  // two fp32 per row (delta, LSE * log2 e), each array 256-byte aligned
   const size_t rows = (size_t)B * H * S;
-  size_t dq = rows * D * sizeof(float);
-  dq = (dq + 255) & ~(size_t)255;
-  return dq + rows * sizeof(float);
+  const size_t one = (rows * sizeof(float) + 255) & ~(size_t)255;
+  return 2 * one;
 }
 
 int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -234,13 +234,13 @@ int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const
   unsigned* err = err_word();
   if (!err) return CPATTN_ERR_CUDA;
   const size_t rows = (size_t)B * H * S;
-  size_t dq_bytes = (rows * D * sizeof(float) + 255) & ~(size_t)255;
-  float* ws_dq = static_cast<float*>(workspace);
-  float* ws_delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + dq_bytes);
+  const size_t one = (rows * sizeof(float) + 255) & ~(size_t)255;
+  float* ws_delta = static_cast<float*>(workspace);
+  float* ws_lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + one);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tc_bwd(sh)) {
     g_last_path = 0;
-    return count(launch_tc_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_dq, ws_delta, err, s));
+    return count(launch_tc_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, s));
   }
   g_last_path = 1;
   return count(launch_simt_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, s));

@@ -41,10 +41,10 @@ int launch_tc_fwd(const AttnShape& sh, const void* q, const void* k, const void*
 int launch_tc_fwd_step(const AttnShape& sh, const void* q, const void* k, const void* v,
                        float* o_part, float* lse_part, int step, unsigned* err,
                        cudaStream_t stream);
-// workspace layout: [dq_acc fp32 B*H*S*D][delta fp32 B*H*S]
+// workspace: per-row delta and LSE * log2(e), fp32 [B*H*S] each
 int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, float* ws_dq, float* ws_delta, unsigned* err, cudaStream_t stream);
+                  void* dv, float* ws_delta, float* ws_lse2, unsigned* err, cudaStream_t stream);
 bool tc_fwd_supported(const AttnShape& sh);
 bool tc_bwd_supported(const AttnShape& sh);
 
@@ -61,8 +61,8 @@ enum KernelId : int {
   kKDelta = 4,
   kKSimtDkdv = 5,
   kKSimtDq = 6,
-  kKTcBwd = 7,
-  kKDqConvert = 8,
+  kKTcDkdv = 7,
+  kKTcDq = 8,
   kKNumKernels = 9
 };
 void prof_begin(int kernel_id, cudaStream_t stream);

@@ -3,31 +3,31 @@
 // Gradient of the ring forward (cpattn_fwd): for every non-SKIP (q chunk, kv
 // chunk) block, recompute P = exp(scale q.k - LSE) from the saved LSE (DIAG
 // blocks masked), then dV += P^T dO, dP = dO V^T, dS = P (dP - delta) with
-// delta_i = dO_i . O_i, dK += scale dS^T Q, dQ += scale dS K.  The walk over
-// q tiles for a given K/V tile mirrors the forward ring: at step t the K/V of
-// rank `owner` sits on rank owner + t ("Megatron-LM source analysis: Context
-// Parallel", section 2: the backward mirrors the forward's exchange; ring rule
-// and zigzag from "Configuring RingAttention+FlashAttention for CP", section 3
-// code and section 5 item 1).
+// delta_i = dO_i . O_i, dK += scale dS^T Q, dQ += scale dS K.
+// ("Megatron-LM source analysis: Context Parallel", section 2: the backward
+// mirrors the forward's exchange; ring rule and zigzag from "Configuring
+// RingAttention+FlashAttention for CP", section 3 code and section 5 item 1.)
 //
-// Launches: (1) preprocess: delta = rowsum(dO * O), zero the fp32 dQ
-// accumulator; (2) the main kernel below; (3) dQ = scale * accumulator -> bf16.
+// Launches:
+//   1. preprocess: delta_i = rowsum(dO_i * O_i), LSE_i * log2(e)   (workspace)
+//   2. dK / dV kernel: one 128-key K/V tile per work item; walks the q tiles
+//      that see it in mirror ring order (at step t the K/V of rank `owner` sits
+//      on rank owner + t): S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T
+//      (bf16, back into TMEM), dV += P^T dO, dK += dS^T Q (A from TMEM).
+//   3. dQ kernel: one 128-row Q tile per work item; walks its K/V tiles in
+//      forward ring order: S = Q K^T, dP = dO V^T, dS (bf16, into TMEM),
+//      dQ += dS K with dQ accumulating in TMEM; written once, no reductions.
+// Splitting dQ out recomputes S and dP once more (7 instead of 5 matrix
+// products per block) but removes the fp32 dQ reduction traffic, which on this
+// GPU costs more than the extra tensor work.
 //
-// Main kernel: persistent, one 128-key K/V tile per work item (longest first).
-// CTA roles (320 threads):
-//   warps 0-3  "softmax": thread = key row (TMEM lane); turns S^T, dP^T into
-//              P^T, dS^T (bf16, written back into TMEM for the dV / dK MMAs)
-//              and dS (into shared memory, the A operand of the dQ MMA);
-//              epilogue of dK, dV
-//   warps 4-7  dQ: thread = query row; reads the dQ tile from TMEM and adds it
-//              into the fp32 accumulator in global memory (vector reductions)
-//   warp  8    TMA: K, V once per item; Q, dO per q tile (two stages)
-//   warp  9    MMA issuer and TMEM owner
-// TMEM (512 columns): S^T [0,128), dP^T [128,256), dV, dK accumulators; for
-// D = 128 the dQ tile (two N = 64 halves) lands in the upper halves of the
-// S^T and dP^T regions, free once P^T and dS^T occupy their lower halves.
-// Per q tile the MMA thread issues S^T, dP^T | dQ | dV, dK, so the dQ read-out
-// overlaps the dV / dK MMAs.
+// Both kernels: persistent, 320 threads.  Warps 0-7 do the elementwise work:
+// warp w owns TMEM lanes 32*(w%4).. (one row per thread) and the column half
+// w/4 of each 128-column score tile.  Warp 8 issues TMA loads, warp 9 the MMAs
+// (one thread) and owns TMEM.  The bf16 P^T / dS^T (dS) values of a column
+// half are packed into the first half of that half's own TMEM columns (half 0
+// -> columns [0,32), half 1 -> [64,96)), so neither half overwrites scores the
+// other is still reading; the MMA k-steps address them accordingly.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,33 +46,6 @@ using namespace sm100;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int D>
-struct BwdCfg {
-  static constexpr int kTileBytes = 128 * D * 2;  // bf16 128-row tile
-  static constexpr int kSubBytes = 128 * 128;     // one 64-column swizzled block
-  static constexpr int kQStages = 2;
-  static constexpr int kThreads = 320;
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;  // stage s: Q at +2s*tile, dO at +(2s+1)*tile
-  static constexpr int kOffDS = kOffQ + kQStages * 2 * kTileBytes;
-  static constexpr int kDSBytes = 128 * 128 * 2;
-  static constexpr int kOffLD = kOffDS + kDSBytes;  // stage s: LSE[128], delta[128] (fp32)
-  static constexpr int kLDBytes = 1024;
-  static constexpr int kOffBar = kOffLD + kQStages * kLDBytes;
-  // no alignment slack: the dynamic shared window starts 1024-byte aligned
-  // (checked at kernel entry)
-  static constexpr int kSmemBytes = kOffBar + 256;
-  static constexpr bool kSplitDq = (D == 128);
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
-  static constexpr uint32_t kColDK = (D == 128) ? 384 : 320;
-  static constexpr uint32_t kColDQ = 384;  // D = 64 only
-  static constexpr int kDqN = kSplitDq ? D / 2 : D;
-  static constexpr uint32_t kIdescST = idesc_bf16_f32(128, 128, 0, 0);
-  static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);
-  static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, kDqN, 1, 1);
-};
-
 struct BwdParams {
   RingGeom g;
   int BH;
@@ -82,15 +55,37 @@ struct BwdParams {
   int G;        // heads per scheduling group (divides BH)
   float sl2;    // scale * log2(e)
   float scale;
-  const float* lse;
-  const float* delta;
-  float* dq_acc;
+  const float* lse2;   // LSE * log2(e), [BH][S]
+  const float* delta;  // [BH][S]
+  __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   unsigned* err;
 };
 
-// Walks, for K/V tile jt, the q tiles that see it in mirror ring order.
+// TMEM column of the packed bf16 pair for score columns (c, c+1) of a tile:
+// column half h = c / 64 packs into [64 h, 64 h + 32).
+__device__ __forceinline__ uint32_t packed_col(int c) { return (c & 64) + ((c & 63) >> 1); }
+// TMEM column of k-step kk (16 score columns) of a packed bf16 operand
+__device__ __forceinline__ uint32_t packed_kstep(int kk) { return (kk >= 4 ? 64 : 0) + (kk & 3) * 8; }
+
+// Work index -> (tile, head).  Heads are taken G at a time so the CTAs busy at
+// any moment share a few heads' operands in L2; inside a group tiles go longest
+// first (ascending K/V position for dK/dV, descending Q position for dQ).
+__device__ __forceinline__ void decode_item(const BwdParams& P, int w, bool descending, int& tile,
+                                            int& bh) {
+  const int per_group = P.G * P.tiles;
+  const int g = w / per_group, r = w % per_group;
+  tile = r / P.G;
+  if (descending) tile = P.tiles - 1 - tile;
+  bh = g * P.G + r % P.G;
+}
+
+__device__ __forceinline__ int snake_item(int round, int cta, int grid) {
+  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+// For K/V tile jt: the q tiles that see it, in mirror ring order.
 struct QIter {
   int b, owner, jt, t, s, it, it_end, diag;
   __device__ __forceinline__ void init(const BwdParams& P, int kv_tile) {
@@ -120,7 +115,6 @@ struct QIter {
       if (it < it_end) return true;
     }
   }
-  // next q tile; is_diag: the q tile shares the K/V tile's positions (mask inside)
   __device__ __forceinline__ bool next(const BwdParams& P, int& qt, int& is_diag) {
     while (it >= it_end)
       if (!next_segment(P)) return false;
@@ -130,71 +124,114 @@ struct QIter {
   }
 };
 
-// Work index -> (K/V tile, head).  Heads are taken G at a time, so the CTAs
-// busy at any moment share a few heads' Q, dO and dQ accumulator in L2; inside
-// a group K/V tiles go in ascending position (most q tiles first).
-__device__ __forceinline__ void decode_item(const BwdParams& P, int w, int& jt, int& bh) {
-  const int per_group = P.G * P.tiles;
-  const int g = w / per_group, r = w % per_group;
-  jt = r / P.G;
-  bh = g * P.G + r % P.G;
+// For Q tile qt: its K/V tiles in forward ring order.
+struct KIter {
+  int a, rank, qt, t, s, kt, kt_end, diag;
+  __device__ __forceinline__ void init(const BwdParams& P, int q_tile) {
+    qt = q_tile;
+    a = qt / P.T;
+    rank = chunk_owner(P.g, a);
+    t = 0;
+    s = -1;
+    kt = kt_end = 0;
+    diag = 0;
+  }
+  __device__ __forceinline__ bool next_segment(const BwdParams& P) {
+    while (true) {
+      ++s;
+      if (s >= slots(P.g)) {
+        s = 0;
+        ++t;
+      }
+      if (t >= P.g.N) return false;
+      const int src = step_src(P.g, rank, t);
+      const int b = rank_chunk(P.g, src, s);
+      const int kind = block_kind(P.g, a, b);
+      if (kind == kSkip) continue;
+      diag = kind == kDiag;
+      kt = b * P.T;
+      kt_end = diag ? qt + 1 : kt + P.T;  // DIAG: K/V tiles up to the q tile's own
+      if (kt < kt_end) return true;
+    }
+  }
+  __device__ __forceinline__ bool next(const BwdParams& P, int& tile, int& is_diag) {
+    while (kt >= kt_end)
+      if (!next_segment(P)) return false;
+    tile = kt++;
+    is_diag = diag && tile == qt;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_scaled(uint32_t a, uint32_t b, float mul) {
+  return pack_bf16x2(__uint_as_float(a) * mul, __uint_as_float(b) * mul);
 }
 
-__device__ __forceinline__ int snake_item(int round, int cta, int grid) {
-  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+// Write 32 fp32 TMEM values (scaled) as bf16 to global memory.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    d4[c] = make_uint4(pack_scaled(v[8 * c], v[8 * c + 1], mul), pack_scaled(v[8 * c + 2], v[8 * c + 3], mul),
+                       pack_scaled(v[8 * c + 4], v[8 * c + 5], mul), pack_scaled(v[8 * c + 6], v[8 * c + 7], mul));
 }
+
+// ===================================================================== dK/dV ==
+template <int D>
+struct DkdvCfg {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kSubBytes = 128 * 128;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;  // stage s: Q at +2s tiles, dO at +(2s+1)
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr int kOffLD = kOffQ + kStages * 2 * kTileBytes;  // stage s: LSE2[128], delta[128]
+  static constexpr int kLDBytes = 1024;
+  static constexpr int kOffBar = kOffLD + kStages * kLDBytes;
+  static constexpr int kSmemBytes = 1024 + kOffBar + 256;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
+  static constexpr uint32_t kColDK = (D == 128) ? 384 : 320;
+  static constexpr uint32_t kIdescST = idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);
+};
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
-    tc_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const __grid_constant__ CUtensorMap tmdQ, const BwdParams P) {
-  using C = BwdCfg<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = smem_raw;
-  if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) atomicOr(P.err, kErrLayout);
-    return;
-  }
+    tc_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                   const BwdParams P) {
+  using C = DkdvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
-  uint8_t* sDS = smem + C::kOffDS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* q_full = bars + 2;   // [2]
-  uint64_t* q_empty = bars + 4;  // [2]
-  uint64_t* s_ready = bars + 6;
-  uint64_t* p_ready = bars + 7;
-  uint64_t* dq_ready = bars + 8;
-  uint64_t* dq_free = bars + 9;
-  uint64_t* kv_done = bars + 10;
-  uint64_t* acc_free = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint64_t* stage_full = bars + 13;  // dQ rows written to the staging tile (128 arrivals)
-  uint64_t* stage_free = bars + 14;  // staging tile read by the TMA reduction
-  uint64_t* ds_free = bars + 15;     // dS buffer free again for the next q tile
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars + 2;             // [kStages]
+  uint64_t* q_empty = q_full + C::kStages;  // [kStages]
+  uint64_t* s_ready = q_empty + C::kStages;
+  uint64_t* p_ready = s_ready + 1;
+  uint64_t* kv_done = s_ready + 2;
+  uint64_t* acc_free = s_ready + 3;
+  uint64_t* drain = s_ready + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_ready + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
     mbar_init(s_ready, 1);
-    mbar_init(p_ready, 128);
-    mbar_init(dq_ready, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(p_ready, 256);
     mbar_init(kv_done, 1);
-    mbar_init(acc_free, 128);
+    mbar_init(acc_free, 256);
     mbar_init(drain, 1);
-    mbar_init(stage_full, 128);
-    mbar_init(stage_free, 1);
-    mbar_init(ds_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -207,7 +244,6 @@ __global__ void __launch_bounds__(320, 1)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
     prefetch_tensormap(&tmdO);
-    prefetch_tensormap(&tmdQ);
   }
   __syncthreads();
   tc_fence_after();
@@ -215,42 +251,37 @@ __global__ void __launch_bounds__(320, 1)
   const int grid = gridDim.x, cta = blockIdx.x;
   const int S = P.g.S;
 
-  if (warp < 4) {
-    // ------------------------------------------------- P^T, dS^T (softmax) --
-    const int rloc = warp * 32 + lane;  // key row within the K/V tile
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  if (warp < 8) {
+    // ---------------------------------------------------- P^T and dS^T --
+    const int quarter = warp & 3, half = warp >> 2;
+    const int rloc = quarter * 32 + lane;  // key row within the K/V tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem_base + lane_off + C::kColS;
     const uint32_t tDP = tmem_base + lane_off + C::kColDP;
-    const uint32_t tDV = tmem_base + lane_off + C::kColDV;
-    const uint32_t tDK = tmem_base + lane_off + C::kColDK;
     uint32_t s_cnt = 0, items = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
       int jt, bh;
-      decode_item(P, w, jt, bh);
+      decode_item(P, w, false, jt, bh);
       QIter qi;
       qi.init(P, jt);
       int qt, dg;
       while (qi.next(P, qt, dg)) {
-        if (!mbar_wait_warp(s_ready, s_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        // the dS buffer doubles as the dQ staging tile of the previous q tile
-        if (s_cnt > 0 && !mbar_wait_warp(ds_free, (s_cnt - 1) & 1, abort_flag, P.err)) {
+        const int st = s_cnt % C::kStages;
+        if (!mbar_wait_warp(s_ready, s_cnt & 1, abort_flag, P.err) ||
+            !mbar_wait_warp(&q_full[st], (s_cnt / C::kStages) & 1, abort_flag, P.err)) {
           ok = false;
           break;
         }
-        // LSE and delta of this q tile arrived with its Q / dO stage
-        if (!mbar_wait_warp(&q_full[s_cnt & 1], (s_cnt >> 1) & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        const float4* lse4 = reinterpret_cast<const float4*>(smem + C::kOffLD + (s_cnt & 1) * C::kLDBytes);
-        const float4* dl4 = lse4 + 32;
         ++s_cnt;
         tc_fence_after();
+        const float4* l4 = reinterpret_cast<const float4*>(smem + C::kOffLD + st * C::kLDBytes);
+        const float4* d4 = l4 + 32;
 #pragma unroll
-        for (int cb = 0; cb < 128; cb += 32) {
+        for (int ch = 0; ch < 2; ++ch) {
+          const int cb = half * 64 + ch * 32;  // first q column of this chunk
           uint32_t sv[32], dpv[32];
           tmem_ld32<0>(tS + cb, sv);
           tmem_ld32<0>(tDP + cb, dpv);
@@ -258,144 +289,50 @@ __global__ void __launch_bounds__(320, 1)
           uint32_t pk[16], dsk[16];
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 L = lse4[(cb >> 2) + c4];
-            const float4 Dl = dl4[(cb >> 2) + c4];
+            const float4 L = l4[(cb >> 2) + c4];
+            const float4 Dl = d4[(cb >> 2) + c4];
             const float lv[4] = {L.x, L.y, L.z, L.w};
-            const float dv_[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
+            const float dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
             float p[4], ds[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int c = cb + 4 * c4 + e;  // q column within the tile
-              float pe = ex2(fmaf(__uint_as_float(sv[4 * c4 + e]), P.sl2, -lv[e] * kLog2e));
-              if (dg && rloc > c) pe = 0.f;  // key after query: masked
+              float pe = ex2(fmaf(__uint_as_float(sv[4 * c4 + e]), P.sl2, -lv[e]));
+              if (dg && rloc > cb + 4 * c4 + e) pe = 0.f;  // key after query: masked
               p[e] = pe;
-              ds[e] = pe * (__uint_as_float(dpv[4 * c4 + e]) - dv_[e]);
+              ds[e] = pe * (__uint_as_float(dpv[4 * c4 + e]) - dl[e]);
             }
             pk[2 * c4] = pack_bf16x2(p[0], p[1]);
             pk[2 * c4 + 1] = pack_bf16x2(p[2], p[3]);
             dsk[2 * c4] = pack_bf16x2(ds[0], ds[1]);
             dsk[2 * c4 + 1] = pack_bf16x2(ds[2], ds[3]);
           }
-          tmem_st16<0>(tS + cb / 2, pk);
-          tmem_st16<0>(tDP + cb / 2, dsk);
-          // dS into shared memory as the MN-major A operand of the dQ MMA:
-          // row = key (K index), 64-query swizzled atoms along M
-          uint8_t* rowp = sDS + (cb >> 6) * C::kSubBytes + rloc * 128;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int chunk = ((cb & 63) >> 3) + u;
-            *reinterpret_cast<uint4*>(rowp + ((chunk ^ (rloc & 7)) << 4)) =
-                make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
-          }
+          tmem_st16<0>(tS + packed_col(cb), pk);
+          tmem_st16<0>(tDP + packed_col(cb), dsk);
         }
         tmem_wait_st();
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_ready);
       }
       if (!ok) break;
-      // epilogue: dV, dK of this K/V tile
+      // epilogue: this warp writes columns [half*D/2, half*D/2 + D/2) of dV, dK
       if (!mbar_wait_warp(kv_done, items & 1, abort_flag, P.err)) break;
       ++items;
       tc_fence_after();
       const long orow = ((long)bh * S + (long)jt * 128 + rloc) * D;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t src = which ? tDK : tDV;
-        const float mul = which ? P.scale : 1.f;
-        __nv_bfloat16* dst = which ? P.dk : P.dv;
-#pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
-          uint32_t ov[32];
-          tmem_ld32<0>(src + cb, ov);
-          tmem_wait_ld();
-          uint4* d4 = reinterpret_cast<uint4*>(dst + orow + cb);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(ov[8 * c + 0]) * mul, __uint_as_float(ov[8 * c + 1]) * mul);
-            u.y = pack_bf16x2(__uint_as_float(ov[8 * c + 2]) * mul, __uint_as_float(ov[8 * c + 3]) * mul);
-            u.z = pack_bf16x2(__uint_as_float(ov[8 * c + 4]) * mul, __uint_as_float(ov[8 * c + 5]) * mul);
-            u.w = pack_bf16x2(__uint_as_float(ov[8 * c + 6]) * mul, __uint_as_float(ov[8 * c + 7]) * mul);
-            d4[c] = u;
-          }
-        }
+      for (int cb = 0; cb < D / 2; cb += 32) {
+        const int col = half * (D / 2) + cb;
+        uint32_t ov[32];
+        tmem_ld32<0>(tmem_base + lane_off + C::kColDV + col, ov);
+        tmem_wait_ld();
+        store_row32(P.dv + orow + col, ov, 1.f);
+        tmem_ld32<0>(tmem_base + lane_off + C::kColDK + col, ov);
+        tmem_wait_ld();
+        store_row32(P.dk + orow + col, ov, P.scale);
       }
       tc_fence_before();
       mbar_arrive(acc_free);
     }
-  } else if (warp < 8) {
-    // -------------------------------------------------- dQ read-out + add --
-    const int quarter = warp - 4;
-    const int rloc = quarter * 32 + lane;  // query row within the q tile
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const bool leader = (quarter == 0);  // warp 4 issues the TMA reductions
-    uint32_t dq_cnt = 0, use_cnt = 0, free_cnt = 0;
-    bool ok = true;
-    for (int round = 0; ok; ++round) {
-      const int w = snake_item(round, cta, grid);
-      if (w >= P.n_items) break;
-      int jt, bh;
-      decode_item(P, w, jt, bh);
-      QIter qi;
-      qi.init(P, jt);
-      int qt, dg;
-      while (qi.next(P, qt, dg)) {
-        if (!mbar_wait_warp(dq_ready, dq_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        ++dq_cnt;
-        tc_fence_after();
-        uint32_t v[D];
-        if constexpr (C::kSplitDq) {
-          tmem_ld32<0>(tmem_base + lane_off + C::kColS + 64, v);
-          tmem_ld32<32>(tmem_base + lane_off + C::kColS + 96, v);
-          tmem_ld32<64>(tmem_base + lane_off + C::kColDP + 64, v);
-          tmem_ld32<96>(tmem_base + lane_off + C::kColDP + 96, v);
-        } else {
-          tmem_ld32<0>(tmem_base + lane_off + C::kColDQ, v);
-          tmem_ld32<32>(tmem_base + lane_off + C::kColDQ + 32, v);
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(dq_free);
-        // Add the tile into the fp32 accumulator with TMA reductions, 64
-        // columns at a time, staged in the dS buffer (free: the dQ MMA that
-        // read it is complete) as two 128-row x 32-column swizzled boxes.
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-          if (h > 0) {
-            if (!mbar_wait_warp(stage_free, free_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-            ++free_cnt;
-          }
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            uint8_t* rowp = sDS + b * C::kSubBytes + rloc * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int col = 64 * h + 32 * b + 4 * c;
-              *reinterpret_cast<uint4*>(rowp + ((c ^ (rloc & 7)) << 4)) =
-                  make_uint4(v[col], v[col + 1], v[col + 2], v[col + 3]);
-            }
-          }
-          fence_proxy_async_smem();
-          mbar_arrive(stage_full);
-          if (leader) {
-            if (!mbar_wait_warp(stage_full, use_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-            if (lane == 0) {
-              const int y = bh * S + qt * 128;
-              tma_reduce_add_2d(&tmdQ, sDS, 64 * h, y);
-              tma_reduce_add_2d(&tmdQ, sDS + C::kSubBytes, 64 * h + 32, y);
-              bulk_commit_group();
-              bulk_wait_read_all();
-              mbar_arrive(h + 1 < D / 64 ? stage_free : ds_free);
-            }
-            __syncwarp();
-          }
-          ++use_cnt;
-        }
-        if (!ok) break;
-      }
-    }
-    if (leader && lane == 0) bulk_wait_all();
   } else if (warp == 8) {
     // ----------------------------------------------------------------- TMA --
     uint32_t items = 0, q_cnt = 0;
@@ -404,7 +341,7 @@ __global__ void __launch_bounds__(320, 1)
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
       int jt, bh;
-      decode_item(P, w, jt, bh);
+      decode_item(P, w, false, jt, bh);
       const int rowbase = bh * S;
       if (items > 0 && !mbar_wait_warp(kv_empty, (items - 1) & 1, abort_flag, P.err)) break;
       if (lane == 0) {
@@ -421,8 +358,9 @@ __global__ void __launch_bounds__(320, 1)
       qi.init(P, jt);
       int qt, dg;
       while (qi.next(P, qt, dg)) {
-        const int st = q_cnt & 1;
-        if (q_cnt >= 2 && !mbar_wait_warp(&q_empty[st], ((q_cnt >> 1) - 1) & 1, abort_flag, P.err)) {
+        const int st = q_cnt % C::kStages;
+        if (q_cnt >= (uint32_t)C::kStages &&
+            !mbar_wait_warp(&q_empty[st], ((q_cnt / C::kStages) - 1) & 1, abort_flag, P.err)) {
           ok = false;
           break;
         }
@@ -437,7 +375,7 @@ __global__ void __launch_bounds__(320, 1)
             tma_load_2d(sdo + sb * C::kSubBytes, &tmdO, &q_full[st], sb * 64, rowbase + qt * 128);
           }
           const long r0 = (long)rowbase + qt * 128;
-          bulk_load(sld, P.lse + r0, 512, &q_full[st]);
+          bulk_load(sld, P.lse2 + r0, 512, &q_full[st]);
           bulk_load(sld + 512, P.delta + r0, 512, &q_full[st]);
         }
         __syncwarp();
@@ -450,22 +388,24 @@ __global__ void __launch_bounds__(320, 1)
       if (items > 0)
         while (!mbar_try_wait(kv_full, (items - 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
         }
-      for (uint32_t i = q_cnt > 2 ? q_cnt - 2 : 0; i < q_cnt; ++i)
-        while (!mbar_try_wait(&q_full[i & 1], (i >> 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
+      const uint32_t first = q_cnt > (uint32_t)C::kStages ? q_cnt - C::kStages : 0;
+      for (uint32_t i = first; i < q_cnt; ++i)
+        while (!mbar_try_wait(&q_full[i % C::kStages], (i / C::kStages) & 1) &&
+               globaltimer() - t0 < kWaitLimitNs) {
         }
     }
   } else {
     // ----------------------------------------------------------------- MMA --
     const uint32_t tS = tmem_base + C::kColS, tDP = tmem_base + C::kColDP;
     const uint32_t tDV = tmem_base + C::kColDV, tDK = tmem_base + C::kColDK;
-    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aDS = smem_u32(sDS);
+    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
     uint32_t items = 0, q_cnt = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
       int jt, bh;
-      decode_item(P, w, jt, bh);
+      decode_item(P, w, false, jt, bh);
       if (!mbar_wait_warp(kv_full, items & 1, abort_flag, P.err)) break;
       tc_fence_after();
       QIter qi;
@@ -473,12 +413,13 @@ __global__ void __launch_bounds__(320, 1)
       int qt, dg;
       bool first = true;
       while (qi.next(P, qt, dg)) {
-        const int st = q_cnt & 1;
+        const int st = q_cnt % C::kStages;
         const uint32_t aQ = smem_u32(smem + C::kOffQ + (2 * st) * C::kTileBytes);
         const uint32_t adO = aQ + C::kTileBytes;
-        if (!mbar_wait_warp(&q_full[st], (q_cnt >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        if (C::kSplitDq && q_cnt > 0 &&
-            !mbar_wait_warp(dq_free, (q_cnt - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        if (!mbar_wait_warp(&q_full[st], (q_cnt / C::kStages) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         if (lane == 0) {
           // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
@@ -498,40 +439,19 @@ __global__ void __launch_bounds__(320, 1)
         }
         __syncwarp();
         if (!mbar_wait_warp(p_ready, q_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        if (!C::kSplitDq && q_cnt > 0 &&
-            !mbar_wait_warp(dq_free, (q_cnt - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
-          // dQ = dS K: A = dS (MN-major, 2 atoms of 64 queries), B = K (MN-major over d)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = smem_desc_sw128(aDS + kk * 2048, C::kSubBytes, 1024);
-            if constexpr (C::kSplitDq) {
-              mma_ss(tS + 64, a, smem_desc_sw128(aK + kk * 2048, C::kSubBytes, 1024), C::kIdescDQ,
-                     kk > 0 ? 1u : 0u);
-              mma_ss(tDP + 64, a, smem_desc_sw128(aK + C::kSubBytes + kk * 2048, C::kSubBytes, 1024),
-                     C::kIdescDQ, kk > 0 ? 1u : 0u);
-            } else {
-              mma_ss(tmem_base + C::kColDQ, a, smem_desc_sw128(aK + kk * 2048, C::kSubBytes, 1024),
-                     C::kIdescDQ, kk > 0 ? 1u : 0u);
-            }
-          }
-          tc_commit(dq_ready);
-        }
-        __syncwarp();
         if (first && items > 0 && !mbar_wait_warp(acc_free, (items - 1) & 1, abort_flag, P.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          // dV += P^T dO, dK += dS^T Q (A from TMEM, B MN-major over d)
+          // dV += P^T dO, dK += dS^T Q (A packed in TMEM, B MN-major over d)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-            mma_ts(tDV, tS + kk * 8, smem_desc_sw128(adO + kk * 2048, C::kSubBytes, 1024),
+            mma_ts(tDV, tS + packed_kstep(kk), smem_desc_sw128(adO + kk * 2048, C::kSubBytes, 1024),
                    C::kIdescAcc, acc);
-            mma_ts(tDK, tDP + kk * 8, smem_desc_sw128(aQ + kk * 2048, C::kSubBytes, 1024),
+            mma_ts(tDK, tDP + packed_kstep(kk), smem_desc_sw128(aQ + kk * 2048, C::kSubBytes, 1024),
                    C::kIdescAcc, acc);
           }
           tc_commit(&q_empty[st]);
@@ -562,12 +482,344 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-// delta_i = sum_d dO_id O_id (fp32) and a zeroed dQ accumulator row; one warp per row
+// ======================================================================== dQ ==
+template <int D>
+struct DqCfg {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kSubBytes = 128 * 128;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kTileBytes;
+  static constexpr int kOffKV = 2 * kTileBytes;  // ring of K / V tiles: K_j, V_j, K_j+1, ...
+  static constexpr int kStages = D == 128 ? 5 : 10;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = 1024 + kOffBar + 256;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColDP = 256, kColDQ = 384;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, 0, 1);
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    tc_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                 const BwdParams P) {
+  using C = DqCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sdO = smem + C::kOffDO;
+  uint8_t* sKV = smem + C::kOffKV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars;                  // [kStages]
+  uint64_t* kv_empty = bars + C::kStages;    // [kStages]
+  uint64_t* q_full = bars + 2 * C::kStages;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* s_ready = q_full + 2;            // [2] one per S buffer
+  uint64_t* dp_ready = q_full + 4;
+  uint64_t* p_ready = q_full + 5;
+  uint64_t* dq_done = q_full + 6;
+  uint64_t* acc_free = q_full + 7;
+  uint64_t* drain = q_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(&s_ready[0], 1);
+    mbar_init(&s_ready[1], 1);
+    mbar_init(dp_ready, 1);
+    mbar_init(p_ready, 256);
+    mbar_init(dq_done, 1);
+    mbar_init(acc_free, 256);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+    prefetch_tensormap(&tmdO);
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int grid = gridDim.x, cta = blockIdx.x;
+  const int S = P.g.S;
+
+  if (warp < 8) {
+    // ------------------------------------------------------------- P, dS --
+    const int quarter = warp & 3, half = warp >> 2;
+    const int rloc = quarter * 32 + lane;  // query row within the Q tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tDP = tmem_base + lane_off + C::kColDP;
+    uint32_t j_cnt = 0, items = 0;
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      const int w = snake_item(round, cta, grid);
+      if (w >= P.n_items) break;
+      int qt, bh;
+      decode_item(P, w, true, qt, bh);
+      const long row = (long)bh * S + (long)qt * 128 + rloc;
+      const float lse2 = P.lse2[row];
+      const float dlt = P.delta[row];
+      KIter ki;
+      ki.init(P, qt);
+      int kt, dg;
+      while (ki.next(P, kt, dg)) {
+        const int sb = j_cnt & 1;
+        const uint32_t tS = tmem_base + lane_off + (sb ? C::kColS1 : C::kColS0);
+        if (!mbar_wait_warp(&s_ready[sb], (j_cnt >> 1) & 1, abort_flag, P.err) ||
+            !mbar_wait_warp(dp_ready, j_cnt & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+        ++j_cnt;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int cb = half * 64 + ch * 32;  // first key column of this chunk
+          uint32_t sv[32], dpv[32];
+          tmem_ld32<0>(tS + cb, sv);
+          tmem_ld32<0>(tDP + cb, dpv);
+          tmem_wait_ld();
+          uint32_t dsk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float p0 = ex2(fmaf(__uint_as_float(sv[c]), P.sl2, -lse2));
+            float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), P.sl2, -lse2));
+            if (dg) {  // key after query: masked
+              if (cb + c > rloc) p0 = 0.f;
+              if (cb + c + 1 > rloc) p1 = 0.f;
+            }
+            dsk[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[c]) - dlt),
+                                      p1 * (__uint_as_float(dpv[c + 1]) - dlt));
+          }
+          tmem_st16<0>(tS + packed_col(cb), dsk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+      }
+      if (!ok) break;
+      // epilogue: dQ columns [half*D/2, half*D/2 + D/2) of this row
+      if (!mbar_wait_warp(dq_done, items & 1, abort_flag, P.err)) break;
+      ++items;
+      tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < D / 2; cb += 32) {
+        const int col = half * (D / 2) + cb;
+        uint32_t ov[32];
+        tmem_ld32<0>(tmem_base + lane_off + C::kColDQ + col, ov);
+        tmem_wait_ld();
+        store_row32(P.dq + row * D + col, ov, P.scale);
+      }
+      tc_fence_before();
+      mbar_arrive(acc_free);
+    }
+  } else if (warp == 8) {
+    // ----------------------------------------------------------------- TMA --
+    uint32_t kv_idx = 0, items = 0;
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      const int w = snake_item(round, cta, grid);
+      if (w >= P.n_items) break;
+      int qt, bh;
+      decode_item(P, w, true, qt, bh);
+      const int rowbase = bh * S;
+      if (items > 0 && !mbar_wait_warp(q_empty, (items - 1) & 1, abort_flag, P.err)) break;
+      if (lane == 0) {
+        mbar_expect_tx(q_full, 2 * C::kTileBytes);
+#pragma unroll
+        for (int sb = 0; sb < D / 64; ++sb) {
+          tma_load_2d(sQ + sb * C::kSubBytes, &tmQ, q_full, sb * 64, rowbase + qt * 128);
+          tma_load_2d(sdO + sb * C::kSubBytes, &tmdO, q_full, sb * 64, rowbase + qt * 128);
+        }
+      }
+      __syncwarp();
+      ++items;
+      KIter ki;
+      ki.init(P, qt);
+      int kt, dg;
+      while (ki.next(P, kt, dg)) {
+        for (int which = 0; which < 2; ++which) {
+          const int s = kv_idx % C::kStages;
+          if (kv_idx >= (uint32_t)C::kStages &&
+              !mbar_wait_warp(&kv_empty[s], ((kv_idx / C::kStages) - 1) & 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_expect_tx(&kv_full[s], C::kTileBytes);
+            const CUtensorMap* map = which ? &tmV : &tmK;
+#pragma unroll
+            for (int sb = 0; sb < D / 64; ++sb)
+              tma_load_2d(sKV + s * C::kTileBytes + sb * C::kSubBytes, map, &kv_full[s], sb * 64,
+                          rowbase + kt * 128);
+          }
+          __syncwarp();
+          ++kv_idx;
+        }
+        if (!ok) break;
+      }
+    }
+    if (*abort_flag) {
+      const unsigned long long t0 = globaltimer();
+      if (items > 0)
+        while (!mbar_try_wait(q_full, (items - 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
+        }
+      const uint32_t first = kv_idx > (uint32_t)C::kStages ? kv_idx - C::kStages : 0;
+      for (uint32_t i = first; i < kv_idx; ++i)
+        while (!mbar_try_wait(&kv_full[i % C::kStages], (i / C::kStages) & 1) &&
+               globaltimer() - t0 < kWaitLimitNs) {
+        }
+    }
+  } else {
+    // ----------------------------------------------------------------- MMA --
+    // Per K/V tile j: S(j+1) is issued before waiting for the elementwise work
+    // of tile j (two S buffers), then dQ += dS(j) K_j and dP(j+1).
+    const uint32_t tDP = tmem_base + C::kColDP, tDQ = tmem_base + C::kColDQ;
+    const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), aKV = smem_u32(sKV);
+    uint32_t kv_idx = 0, j_cnt = 0, items = 0;
+    bool ok = true;
+    auto issue_s = [&](uint32_t sbuf, uint32_t slotK) {
+      const uint32_t tS = tmem_base + (sbuf ? C::kColS1 : C::kColS0);
+      const uint32_t kb = aKV + slotK * C::kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+        mma_ss(tS, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+               C::kIdescS, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_dp = [&](uint32_t slotV) {
+      const uint32_t vb = aKV + slotV * C::kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+        mma_ss(tDP, smem_desc_sw128(adO + off, 16, 1024), smem_desc_sw128(vb + off, 16, 1024),
+               C::kIdescS, kk > 0 ? 1u : 0u);
+      }
+    };
+    for (int round = 0; ok; ++round) {
+      const int w = snake_item(round, cta, grid);
+      if (w >= P.n_items) break;
+      int qt, bh;
+      decode_item(P, w, true, qt, bh);
+      if (!mbar_wait_warp(q_full, items & 1, abort_flag, P.err)) break;
+      tc_fence_after();
+      KIter ki;
+      ki.init(P, qt);
+      int kt, dg;
+      // prologue: S(0), dP(0)
+      if (!ki.next(P, kt, dg)) break;  // unreachable: a q tile always sees its own block
+      uint32_t sK = kv_idx % C::kStages, phK = (kv_idx / C::kStages) & 1;
+      uint32_t sV = (kv_idx + 1) % C::kStages, phV = ((kv_idx + 1) / C::kStages) & 1;
+      kv_idx += 2;
+      if (!mbar_wait_warp(&kv_full[sK], phK, abort_flag, P.err)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        issue_s(j_cnt & 1, sK);
+        tc_commit(&s_ready[j_cnt & 1]);
+      }
+      __syncwarp();
+      if (!mbar_wait_warp(&kv_full[sV], phV, abort_flag, P.err)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        issue_dp(sV);
+        tc_commit(dp_ready);
+        tc_commit(&kv_empty[sV]);
+      }
+      __syncwarp();
+      bool first = true;
+      while (true) {
+        // S(j+1) into the other buffer, overlapping the elementwise work of j
+        const bool more = ki.next(P, kt, dg);
+        uint32_t sK2 = 0, sV2 = 0, phV2 = 0;
+        if (more) {
+          sK2 = kv_idx % C::kStages;
+          const uint32_t phK2 = (kv_idx / C::kStages) & 1;
+          sV2 = (kv_idx + 1) % C::kStages;
+          phV2 = ((kv_idx + 1) / C::kStages) & 1;
+          kv_idx += 2;
+          if (!mbar_wait_warp(&kv_full[sK2], phK2, abort_flag, P.err)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            issue_s((j_cnt + 1) & 1, sK2);
+            tc_commit(&s_ready[(j_cnt + 1) & 1]);
+          }
+          __syncwarp();
+        }
+        if (!mbar_wait_warp(p_ready, j_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+        if (first && items > 0 && !mbar_wait_warp(acc_free, (items - 1) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          // dQ += dS(j) K_j: A = dS packed in the S buffer, B = K_j MN-major over d
+          const uint32_t tS = tmem_base + ((j_cnt & 1) ? C::kColS1 : C::kColS0);
+          const uint32_t kb = aKV + sK * C::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tDQ, tS + packed_kstep(kk), smem_desc_sw128(kb + kk * 2048, C::kSubBytes, 1024),
+                   C::kIdescDQ, (first && kk == 0) ? 0u : 1u);
+          tc_commit(&kv_empty[sK]);
+        }
+        __syncwarp();
+        first = false;
+        ++j_cnt;
+        if (!more) break;
+        if (!mbar_wait_warp(&kv_full[sV2], phV2, abort_flag, P.err)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {
+          issue_dp(sV2);
+          tc_commit(dp_ready);
+          tc_commit(&kv_empty[sV2]);
+        }
+        __syncwarp();
+        sK = sK2;
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        tc_commit(q_empty);  // every S / dP of this Q tile has been issued
+        tc_commit(dq_done);
+      }
+      __syncwarp();
+      ++items;
+    }
+    if (lane == 0) tc_commit(drain);
+    __syncwarp();
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// delta_i = sum_d dO_id O_id and LSE_i * log2(e); one warp per row
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout,
+                                                      const float* __restrict__ lse,
                                                       float* __restrict__ delta,
-                                                      float* __restrict__ dq_acc, long rows) {
+                                                      float* __restrict__ lse2, long rows) {
   const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -584,44 +836,37 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) delta[row] = acc;
-  float* z = dq_acc + row * D + lane * E;
-#pragma unroll
-  for (int e = 0; e < E; e += 2) *reinterpret_cast<float2*>(z + e) = make_float2(0.f, 0.f);
+  if (lane == 0) {
+    delta[row] = acc;
+    lse2[row] = lse[row] * kLog2e;
+  }
 }
 
-// dq = bf16(scale * dq_acc), four elements per thread-iteration
-__global__ void dq_convert_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq, float scale,
-                                  long n4) {
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4;
-       i += (long)gridDim.x * blockDim.x) {
-    const float4 x = acc[i];
-    uint2 u;
-    u.x = pack_bf16x2(x.x * scale, x.y * scale);
-    u.y = pack_bf16x2(x.z * scale, x.w * scale);
-    dq[i] = u;
-  }
+template <typename Cfg, typename Kern>
+bool set_smem(Kern kern, bool& done) {
+  if (done) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+      cudaSuccess)
+    return false;
+  done = true;
+  return true;
 }
 
 template <int D>
 int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v, const void* o,
-                const float* lse, const void* dout, void* dq, void* dk, void* dv, float* ws_dq,
-                float* ws_delta, unsigned* err, cudaStream_t stream) {
-  using C = BwdCfg<D>;
+                const float* lse, const void* dout, void* dq, void* dk, void* dv, float* ws_delta,
+                float* ws_lse2, unsigned* err, cudaStream_t stream) {
   const long rows = (long)sh.B * sh.H * sh.S;
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo;
   if (!make_tmap_bf16_2d(&mq, q, rows, D, 64, 128) || !make_tmap_bf16_2d(&mk, k, rows, D, 64, 128) ||
-      !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128) || !make_tmap_bf16_2d(&mdo, dout, rows, D, 64, 128) ||
-      !make_tmap_f32_2d(&mdq, ws_dq, rows, D, 32, 128))
+      !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128) || !make_tmap_bf16_2d(&mdo, dout, rows, D, 64, 128))
     return -1;
-  int launched = 0;
   prof_begin(kKDelta, stream);
   bwd_pre_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), ws_delta, ws_dq,
-      rows);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, ws_delta,
+      ws_lse2, rows);
   prof_end(kKDelta, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
-  ++launched;
 
   BwdParams P;
   P.g = sh.g;
@@ -632,39 +877,29 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.G = (P.BH % 2 == 0) ? 2 : 1;
   P.sl2 = sh.scale * kLog2e;
   P.scale = sh.scale;
-  P.lse = lse;
+  P.lse2 = ws_lse2;
   P.delta = ws_delta;
-  P.dq_acc = ws_dq;
+  P.dq = static_cast<__nv_bfloat16*>(dq);
   P.dk = static_cast<__nv_bfloat16*>(dk);
   P.dv = static_cast<__nv_bfloat16*>(dv);
   P.err = err;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[D == 128]) {
-    if (cudaFuncSetAttribute(tc_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return -1;
-    attr_set[D == 128] = true;
-  }
+  static bool attr_dkdv[2] = {false, false}, attr_dq[2] = {false, false};
+  if (!set_smem<DkdvCfg<D>>(tc_dkdv_kernel<D>, attr_dkdv[D == 128]) ||
+      !set_smem<DqCfg<D>>(tc_dq_kernel<D>, attr_dq[D == 128]))
+    return -1;
   int dev = 0;
   cudaGetDevice(&dev);
   int grid = num_sms(dev);
   if (grid > P.n_items) grid = P.n_items;
-  prof_begin(kKTcBwd, stream);
-  tc_bwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, P);
-  prof_end(kKTcBwd, stream);
+  prof_begin(kKTcDkdv, stream);
+  tc_dkdv_kernel<D><<<grid, 320, DkdvCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
+  prof_end(kKTcDkdv, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
-  ++launched;
-
-  const long n4 = rows * D / 4;
-  long blocks = (n4 + 255) / 256;
-  if (blocks > 148L * 16) blocks = 148L * 16;
-  prof_begin(kKDqConvert, stream);
-  dq_convert_kernel<<<(unsigned)blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(ws_dq),
-                                                          reinterpret_cast<uint2*>(dq), sh.scale, n4);
-  prof_end(kKDqConvert, stream);
+  prof_begin(kKTcDq, stream);
+  tc_dq_kernel<D><<<grid, 320, DqCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
+  prof_end(kKTcDq, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
-  ++launched;
-  return launched;
+  return 3;
 }
 
 }  // namespace
@@ -679,10 +914,10 @@ bool tc_bwd_supported(const AttnShape& sh) {
 
 int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, float* ws_dq, float* ws_delta, unsigned* err, cudaStream_t stream) {
+                  void* dv, float* ws_delta, float* ws_lse2, unsigned* err, cudaStream_t stream) {
   if (sh.D == 64)
-    return launch_impl<64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_dq, ws_delta, err, stream);
-  return launch_impl<128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_dq, ws_delta, err, stream);
+    return launch_impl<64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
+  return launch_impl<128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
 }
 
 }  // namespace cpattn

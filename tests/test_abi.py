@@ -90,7 +90,7 @@ def test_argument_errors_are_reported_before_launch(cp):
     assert cp.lib.cpattn_finalize(p, p, 10, 128, 5, None) == cp.ERR_DTYPE
     # backward: workspace checks
     need = cp.bwd_workspace_bytes(1, 1, 256, 128)
-    assert need >= 256 * 128 * 4 + 256 * 4
+    assert need >= 2 * 256 * 4
     args = [p] * 9 + [1, 1, 256, 128, 2, 1, 0.1]
     assert cp.lib.cpattn_bwd(*args, None, need, 0, None) == cp.ERR_WORKSPACE
     assert cp.lib.cpattn_bwd(*args, p, need - 1, 0, None) == cp.ERR_WORKSPACE
