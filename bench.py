@@ -119,13 +119,20 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(x, world):
+    """Largest value of x over all ranks (the job's time is its slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tflops(flops_per_rank_step, steps, ms_max, world):
+    """Whole-job throughput: every rank runs its own replica of the workload."""
+    return world * flops_per_rank_step * steps / (ms_max * 1e-3) / 1e12
 
 
 def barrier(world):
@@ -259,7 +266,7 @@ def run_gpu(args, w):
 
     ms_step = ms_total / args.steps
     f_fwd, f_bwd = w.flops_fwd(), (0.0 if args.fwd_only else w.flops_bwd())
-    value = world * (f_fwd + f_bwd) * args.steps / (ms_total * 1e-3) / 1e12
+    value = job_tflops(f_fwd + f_bwd, args.steps, ms_total, world)
 
     per_kernel = {}
     for kind, name in cp.KERNEL_KINDS.items():
@@ -313,7 +320,7 @@ def run_gpu(args, w):
         torch.cuda.synchronize(dev)
         barrier(world)
         e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
-        e2e = {"value": world * (f_fwd + f_bwd) * n_e2e / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_tflops(f_fwd + f_bwd, n_e2e, e2e_ms, world), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": e2e_ms / n_e2e}
 
