@@ -1,4 +1,6 @@
-// tc_bwd.cu -- tcgen05 tensor-core recompute backward for bf16, D in {64,128}.
+// tc_bwd.cu -- tcgen05 tensor-core recompute backward for bf16, D in {64,128}:
+// the preprocess, the dK / dV kernel and the launch sequence (the dQ kernel is
+// in tc_dq.cu).
 //
 // Gradient of the ring forward (cpattn_fwd): for every non-SKIP (q chunk, kv
 // chunk) block, recompute P = exp(scale q.k - LSE) from the saved LSE (DIAG
@@ -14,19 +16,18 @@
 //      that see it in mirror ring order (at step t the K/V of rank `owner` sits
 //      on rank owner + t): S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T
 //      (bf16, back into TMEM), dV += P^T dO, dK += dS^T Q (A from TMEM).
-//   3. dQ kernel: one 128-row Q tile per work item; walks its K/V tiles in
-//      forward ring order: S = Q K^T, dP = dO V^T, dS (bf16, into TMEM),
-//      dQ += dS K with dQ accumulating in TMEM; written once, no reductions.
-// Splitting dQ out recomputes S and dP once more (7 instead of 5 matrix
-// products per block) but removes the fp32 dQ reduction traffic, which on this
-// GPU costs more than the extra tensor work.
+//   3. dQ kernel (tc_dq.cu): one Q tile per work item, dQ accumulated in TMEM
+//      and written once; no reductions.
+// Computing dQ in its own kernel recomputes S and dP once more but removes the
+// fp32 dQ reduction traffic, which on this GPU costs more than the extra
+// tensor work.
 //
-// Both kernels: persistent, 320 threads.  Warps 0-7 do the elementwise work:
-// warp w owns TMEM lanes 32*(w%4).. (one row per thread) and the column half
-// w/4 of each 128-column score tile.  Warp 8 issues TMA loads, warp 9 the MMAs
-// (one thread) and owns TMEM.  The bf16 P^T / dS^T (dS) values of a column
-// half are packed into the first half of that half's own TMEM columns (half 0
-// -> columns [0,32), half 1 -> [64,96)), so neither half overwrites scores the
+// dK / dV kernel: persistent, 320 threads.  Warps 0-7 do the elementwise work:
+// warp w owns TMEM lanes 32*(w%4).. (one key row per thread) and the column
+// half w/4 of each 128-column score tile.  Warp 8 issues TMA loads, warp 9 the
+// MMAs (one thread) and owns TMEM.  The bf16 P^T / dS^T values of a column half
+// are packed into the first half of that half's own TMEM columns (half 0 ->
+// columns [0,32), half 1 -> [64,96)), so neither half overwrites scores the
 // other is still reading; the MMA k-steps address them accordingly.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -34,11 +35,17 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "bwd_common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 #include "tmap.h"
 
 namespace cpattn {
+namespace bwd {
+
+template <int D>
+int launch_tc_dq(const BwdParams& P, const CUtensorMap& mq, const CUtensorMap& mk,
+                 const CUtensorMap& mv, const CUtensorMap& mdo, int grid, cudaStream_t stream);
 
 namespace {
 
@@ -46,135 +53,11 @@ using namespace sm100;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-struct BwdParams {
-  RingGeom g;
-  int BH;
-  int T;        // 128-row tiles per chunk
-  int tiles;    // 128-row tiles per head (S / 128)
-  int n_items;  // BH * tiles
-  int G;        // heads per scheduling group (divides BH)
-  float sl2;    // scale * log2(e)
-  float scale;
-  const float* lse2;   // LSE * log2(e), [BH][S]
-  const float* delta;  // [BH][S]
-  __nv_bfloat16* dq;
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
-  unsigned* err;
-};
-
 // TMEM column of the packed bf16 pair for score columns (c, c+1) of a tile:
 // column half h = c / 64 packs into [64 h, 64 h + 32).
 __device__ __forceinline__ uint32_t packed_col(int c) { return (c & 64) + ((c & 63) >> 1); }
 // TMEM column of k-step kk (16 score columns) of a packed bf16 operand
 __device__ __forceinline__ uint32_t packed_kstep(int kk) { return (kk >= 4 ? 64 : 0) + (kk & 3) * 8; }
-
-// Work index -> (tile, head).  Heads are taken G at a time so the CTAs busy at
-// any moment share a few heads' operands in L2; inside a group tiles go longest
-// first (ascending K/V position for dK/dV, descending Q position for dQ).
-__device__ __forceinline__ void decode_item(const BwdParams& P, int w, bool descending, int& tile,
-                                            int& bh) {
-  const int per_group = P.G * P.tiles;
-  const int g = w / per_group, r = w % per_group;
-  tile = r / P.G;
-  if (descending) tile = P.tiles - 1 - tile;
-  bh = g * P.G + r % P.G;
-}
-
-__device__ __forceinline__ int snake_item(int round, int cta, int grid) {
-  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
-}
-
-// For K/V tile jt: the q tiles that see it, in mirror ring order.
-struct QIter {
-  int b, owner, jt, t, s, it, it_end, diag;
-  __device__ __forceinline__ void init(const BwdParams& P, int kv_tile) {
-    jt = kv_tile;
-    b = jt / P.T;
-    owner = chunk_owner(P.g, b);
-    t = 0;
-    s = -1;
-    it = it_end = 0;
-    diag = 0;
-  }
-  __device__ __forceinline__ bool next_segment(const BwdParams& P) {
-    while (true) {
-      ++s;
-      if (s >= slots(P.g)) {
-        s = 0;
-        ++t;
-      }
-      if (t >= P.g.N) return false;
-      const int r = (owner + t) % P.g.N;  // rank holding this K/V at step t
-      const int a = rank_chunk(P.g, r, s);
-      const int kind = block_kind(P.g, a, b);
-      if (kind == kSkip) continue;
-      diag = kind == kDiag;
-      it = diag ? jt : a * P.T;  // in a DIAG block only q tiles at or after jt see it
-      it_end = (a + 1) * P.T;
-      if (it < it_end) return true;
-    }
-  }
-  __device__ __forceinline__ bool next(const BwdParams& P, int& qt, int& is_diag) {
-    while (it >= it_end)
-      if (!next_segment(P)) return false;
-    qt = it++;
-    is_diag = diag && qt == jt;
-    return true;
-  }
-};
-
-// For Q tile qt: its K/V tiles in forward ring order.
-struct KIter {
-  int a, rank, qt, t, s, kt, kt_end, diag;
-  __device__ __forceinline__ void init(const BwdParams& P, int q_tile) {
-    qt = q_tile;
-    a = qt / P.T;
-    rank = chunk_owner(P.g, a);
-    t = 0;
-    s = -1;
-    kt = kt_end = 0;
-    diag = 0;
-  }
-  __device__ __forceinline__ bool next_segment(const BwdParams& P) {
-    while (true) {
-      ++s;
-      if (s >= slots(P.g)) {
-        s = 0;
-        ++t;
-      }
-      if (t >= P.g.N) return false;
-      const int src = step_src(P.g, rank, t);
-      const int b = rank_chunk(P.g, src, s);
-      const int kind = block_kind(P.g, a, b);
-      if (kind == kSkip) continue;
-      diag = kind == kDiag;
-      kt = b * P.T;
-      kt_end = diag ? qt + 1 : kt + P.T;  // DIAG: K/V tiles up to the q tile's own
-      if (kt < kt_end) return true;
-    }
-  }
-  __device__ __forceinline__ bool next(const BwdParams& P, int& tile, int& is_diag) {
-    while (kt >= kt_end)
-      if (!next_segment(P)) return false;
-    tile = kt++;
-    is_diag = diag && tile == qt;
-    return true;
-  }
-};
-
-__device__ __forceinline__ uint32_t pack_scaled(uint32_t a, uint32_t b, float mul) {
-  return pack_bf16x2(__uint_as_float(a) * mul, __uint_as_float(b) * mul);
-}
-
-// Write 32 fp32 TMEM values (scaled) as bf16 to global memory.
-__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    d4[c] = make_uint4(pack_scaled(v[8 * c], v[8 * c + 1], mul), pack_scaled(v[8 * c + 2], v[8 * c + 3], mul),
-                       pack_scaled(v[8 * c + 4], v[8 * c + 5], mul), pack_scaled(v[8 * c + 6], v[8 * c + 7], mul));
-}
 
 // ===================================================================== dK/dV ==
 template <int D>
@@ -211,12 +94,14 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* kv_empty = bars + 1;
   uint64_t* q_full = bars + 2;             // [kStages]
   uint64_t* q_empty = q_full + C::kStages;  // [kStages]
-  uint64_t* s_ready = q_empty + C::kStages;
-  uint64_t* p_ready = s_ready + 1;
-  uint64_t* kv_done = s_ready + 2;
-  uint64_t* acc_free = s_ready + 3;
-  uint64_t* drain = s_ready + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_ready + 5);
+  uint64_t* s_ready = q_empty + C::kStages;  // S^T of the q tile in TMEM
+  uint64_t* dp_ready = s_ready + 1;          // dP^T of the q tile in TMEM
+  uint64_t* pa_ready = s_ready + 2;          // P^T written back (256 arrivals)
+  uint64_t* pb_ready = s_ready + 3;          // dS^T written back (256 arrivals)
+  uint64_t* kv_done = s_ready + 4;
+  uint64_t* acc_free = s_ready + 5;
+  uint64_t* drain = s_ready + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_ready + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -228,7 +113,9 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&q_empty[i], 1);
     }
     mbar_init(s_ready, 1);
-    mbar_init(p_ready, 256);
+    mbar_init(dp_ready, 1);
+    mbar_init(pa_ready, 256);
+    mbar_init(pb_ready, 256);
     mbar_init(kv_done, 1);
     mbar_init(acc_free, 256);
     mbar_init(drain, 1);
@@ -270,48 +157,66 @@ __global__ void __launch_bounds__(320, 1)
       int qt, dg;
       while (qi.next(P, qt, dg)) {
         const int st = s_cnt % C::kStages;
+        // exponential phase: needs S^T only; P^T goes back to TMEM for dV
         if (!mbar_wait_warp(s_ready, s_cnt & 1, abort_flag, P.err) ||
             !mbar_wait_warp(&q_full[st], (s_cnt / C::kStages) & 1, abort_flag, P.err)) {
           ok = false;
           break;
         }
-        ++s_cnt;
         tc_fence_after();
         const float4* l4 = reinterpret_cast<const float4*>(smem + C::kOffLD + st * C::kLDBytes);
         const float4* d4 = l4 + 32;
+        float p[64];
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           const int cb = half * 64 + ch * 32;  // first q column of this chunk
-          uint32_t sv[32], dpv[32];
+          uint32_t sv[32], pk[16];
           tmem_ld32<0>(tS + cb, sv);
-          tmem_ld32<0>(tDP + cb, dpv);
           tmem_wait_ld();
-          uint32_t pk[16], dsk[16];
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
             const float4 L = l4[(cb >> 2) + c4];
-            const float4 Dl = d4[(cb >> 2) + c4];
             const float lv[4] = {L.x, L.y, L.z, L.w};
-            const float dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
-            float p[4], ds[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float pe = ex2(fmaf(__uint_as_float(sv[4 * c4 + e]), P.sl2, -lv[e]));
               if (dg && rloc > cb + 4 * c4 + e) pe = 0.f;  // key after query: masked
-              p[e] = pe;
-              ds[e] = pe * (__uint_as_float(dpv[4 * c4 + e]) - dl[e]);
+              p[ch * 32 + 4 * c4 + e] = pe;
             }
-            pk[2 * c4] = pack_bf16x2(p[0], p[1]);
-            pk[2 * c4 + 1] = pack_bf16x2(p[2], p[3]);
+            pk[2 * c4] = pack_bf16x2(p[ch * 32 + 4 * c4], p[ch * 32 + 4 * c4 + 1]);
+            pk[2 * c4 + 1] = pack_bf16x2(p[ch * 32 + 4 * c4 + 2], p[ch * 32 + 4 * c4 + 3]);
+          }
+          tmem_st16<0>(tS + packed_col(cb), pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(pa_ready);
+        // dS phase: needs dP^T; dS^T goes back to TMEM for dK
+        if (!mbar_wait_warp(dp_ready, s_cnt & 1, abort_flag, P.err)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const int cb = half * 64 + ch * 32;
+          uint32_t dpv[32], dsk[16];
+          tmem_ld32<0>(tDP + cb, dpv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 Dl = d4[(cb >> 2) + c4];
+            const float dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
+            float ds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              ds[e] = p[ch * 32 + 4 * c4 + e] * (__uint_as_float(dpv[4 * c4 + e]) - dl[e]);
             dsk[2 * c4] = pack_bf16x2(ds[0], ds[1]);
             dsk[2 * c4 + 1] = pack_bf16x2(ds[2], ds[3]);
           }
-          tmem_st16<0>(tS + packed_col(cb), pk);
           tmem_st16<0>(tDP + packed_col(cb), dsk);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_ready);
+        mbar_arrive(pb_ready);
       }
       if (!ok) break;
       // epilogue: this warp writes columns [half*D/2, half*D/2 + D/2) of dV, dK
@@ -401,400 +306,99 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
     uint32_t items = 0, q_cnt = 0;
     bool ok = true;
+    auto q_addr = [&](uint32_t cnt) {
+      return smem_u32(smem + C::kOffQ + (2 * (cnt % C::kStages)) * C::kTileBytes);
+    };
+    // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+    auto issue_st = [&](uint32_t aQ) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+        mma_ss(tS, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
+               C::kIdescST, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_dpt = [&](uint32_t adO) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+        mma_ss(tDP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
+               C::kIdescST, kk > 0 ? 1u : 0u);
+      }
+    };
+    // Per q tile t the order is dV(t), S^T(t+1), dK(t), dP^T(t+1): dV(t) and
+    // S^T(t+1) run under the dS phase of t, dK(t) and dP^T(t+1) under the
+    // exponential phase of t+1.
     for (int round = 0; ok; ++round) {
       const int w = snake_item(round, cta, grid);
       if (w >= P.n_items) break;
       int jt, bh;
       decode_item(P, w, false, jt, bh);
-      if (!mbar_wait_warp(kv_full, items & 1, abort_flag, P.err)) break;
-      tc_fence_after();
       QIter qi;
       qi.init(P, jt);
-      int qt, dg;
-      bool first = true;
-      while (qi.next(P, qt, dg)) {
-        const int st = q_cnt % C::kStages;
-        const uint32_t aQ = smem_u32(smem + C::kOffQ + (2 * st) * C::kTileBytes);
-        const uint32_t adO = aQ + C::kTileBytes;
-        if (!mbar_wait_warp(&q_full[st], (q_cnt / C::kStages) & 1, abort_flag, P.err)) {
+      int n = 0, qt, dg;
+      while (qi.next(P, qt, dg)) ++n;
+      const uint32_t base = q_cnt;
+      q_cnt += n;
+      if (!mbar_wait_warp(kv_full, items & 1, abort_flag, P.err) ||
+          !mbar_wait_warp(&q_full[base % C::kStages], (base / C::kStages) & 1, abort_flag, P.err))
+        break;
+      tc_fence_after();
+      if (lane == 0) {
+        issue_st(q_addr(base));
+        tc_commit(s_ready);
+        issue_dpt(q_addr(base) + C::kTileBytes);
+        tc_commit(dp_ready);
+      }
+      __syncwarp();
+      for (int t = 0; t < n; ++t) {
+        const uint32_t cnt = base + t;
+        const uint32_t aQ = q_addr(cnt), adO = aQ + C::kTileBytes;
+        if (!mbar_wait_warp(pa_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
+        if (t == 0 && items > 0 && !mbar_wait_warp(acc_free, (items - 1) & 1, abort_flag, P.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
-          // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+        if (lane == 0) {  // dV += P^T dO (A packed in TMEM, B MN-major over d)
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-            mma_ss(tS, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
-                   C::kIdescST, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-            mma_ss(tDP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
-                   C::kIdescST, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(s_ready);
-        }
-        __syncwarp();
-        if (!mbar_wait_warp(p_ready, q_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        if (first && items > 0 && !mbar_wait_warp(acc_free, (items - 1) & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          // dV += P^T dO, dK += dS^T Q (A packed in TMEM, B MN-major over d)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          for (int kk = 0; kk < 8; ++kk)
             mma_ts(tDV, tS + packed_kstep(kk), smem_desc_sw128(adO + kk * 2048, C::kSubBytes, 1024),
-                   C::kIdescAcc, acc);
-            mma_ts(tDK, tDP + packed_kstep(kk), smem_desc_sw128(aQ + kk * 2048, C::kSubBytes, 1024),
-                   C::kIdescAcc, acc);
-          }
-          tc_commit(&q_empty[st]);
+                   C::kIdescAcc, (t == 0 && kk == 0) ? 0u : 1u);
         }
         __syncwarp();
-        first = false;
-        ++q_cnt;
+        if (t + 1 < n) {
+          if (!mbar_wait_warp(&q_full[(cnt + 1) % C::kStages], ((cnt + 1) / C::kStages) & 1, abort_flag,
+                              P.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            issue_st(q_addr(cnt + 1));
+            tc_commit(s_ready);
+          }
+          __syncwarp();
+        }
+        if (!mbar_wait_warp(pb_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
+        tc_fence_after();
+        if (lane == 0) {  // dK += dS^T Q
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tDK, tDP + packed_kstep(kk), smem_desc_sw128(aQ + kk * 2048, C::kSubBytes, 1024),
+                   C::kIdescAcc, (t == 0 && kk == 0) ? 0u : 1u);
+          tc_commit(&q_empty[cnt % C::kStages]);
+          if (t + 1 < n) {
+            issue_dpt(q_addr(cnt + 1) + C::kTileBytes);
+            tc_commit(dp_ready);
+          }
+        }
+        __syncwarp();
       }
       if (!ok) break;
       if (lane == 0) {
         tc_commit(kv_empty);
         tc_commit(kv_done);
-      }
-      __syncwarp();
-      ++items;
-    }
-    if (lane == 0) tc_commit(drain);
-    __syncwarp();
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
-    }
-  }
-
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
-  }
-}
-
-// ======================================================================== dQ ==
-template <int D>
-struct DqCfg {
-  static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kSubBytes = 128 * 128;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffDO = kTileBytes;
-  static constexpr int kOffKV = 2 * kTileBytes;  // ring of K / V tiles: K_j, V_j, K_j+1, ...
-  static constexpr int kStages = D == 128 ? 5 : 10;
-  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kSmemBytes = 1024 + kOffBar + 256;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColDP = 256, kColDQ = 384;
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
-  static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, 0, 1);
-};
-
-template <int D>
-__global__ void __launch_bounds__(320, 1)
-    tc_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                 const BwdParams P) {
-  using C = DqCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* sQ = smem + C::kOffQ;
-  uint8_t* sdO = smem + C::kOffDO;
-  uint8_t* sKV = smem + C::kOffKV;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_full = bars;                  // [kStages]
-  uint64_t* kv_empty = bars + C::kStages;    // [kStages]
-  uint64_t* q_full = bars + 2 * C::kStages;
-  uint64_t* q_empty = q_full + 1;
-  uint64_t* s_ready = q_full + 2;            // [2] one per S buffer
-  uint64_t* dp_ready = q_full + 4;
-  uint64_t* p_ready = q_full + 5;
-  uint64_t* dq_done = q_full + 6;
-  uint64_t* acc_free = q_full + 7;
-  uint64_t* drain = q_full + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 9);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    mbar_init(&s_ready[0], 1);
-    mbar_init(&s_ready[1], 1);
-    mbar_init(dp_ready, 1);
-    mbar_init(p_ready, 256);
-    mbar_init(dq_done, 1);
-    mbar_init(acc_free, 256);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 9) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  if (warp == 8 && lane == 0) {
-    prefetch_tensormap(&tmQ);
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-    prefetch_tensormap(&tmdO);
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const int grid = gridDim.x, cta = blockIdx.x;
-  const int S = P.g.S;
-
-  if (warp < 8) {
-    // ------------------------------------------------------------- P, dS --
-    const int quarter = warp & 3, half = warp >> 2;
-    const int rloc = quarter * 32 + lane;  // query row within the Q tile
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tDP = tmem_base + lane_off + C::kColDP;
-    uint32_t j_cnt = 0, items = 0;
-    bool ok = true;
-    for (int round = 0; ok; ++round) {
-      const int w = snake_item(round, cta, grid);
-      if (w >= P.n_items) break;
-      int qt, bh;
-      decode_item(P, w, true, qt, bh);
-      const long row = (long)bh * S + (long)qt * 128 + rloc;
-      const float lse2 = P.lse2[row];
-      const float dlt = P.delta[row];
-      KIter ki;
-      ki.init(P, qt);
-      int kt, dg;
-      while (ki.next(P, kt, dg)) {
-        const int sb = j_cnt & 1;
-        const uint32_t tS = tmem_base + lane_off + (sb ? C::kColS1 : C::kColS0);
-        if (!mbar_wait_warp(&s_ready[sb], (j_cnt >> 1) & 1, abort_flag, P.err) ||
-            !mbar_wait_warp(dp_ready, j_cnt & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        ++j_cnt;
-        tc_fence_after();
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const int cb = half * 64 + ch * 32;  // first key column of this chunk
-          uint32_t sv[32], dpv[32];
-          tmem_ld32<0>(tS + cb, sv);
-          tmem_ld32<0>(tDP + cb, dpv);
-          tmem_wait_ld();
-          uint32_t dsk[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float p0 = ex2(fmaf(__uint_as_float(sv[c]), P.sl2, -lse2));
-            float p1 = ex2(fmaf(__uint_as_float(sv[c + 1]), P.sl2, -lse2));
-            if (dg) {  // key after query: masked
-              if (cb + c > rloc) p0 = 0.f;
-              if (cb + c + 1 > rloc) p1 = 0.f;
-            }
-            dsk[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dpv[c]) - dlt),
-                                      p1 * (__uint_as_float(dpv[c + 1]) - dlt));
-          }
-          tmem_st16<0>(tS + packed_col(cb), dsk);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_ready);
-      }
-      if (!ok) break;
-      // epilogue: dQ columns [half*D/2, half*D/2 + D/2) of this row
-      if (!mbar_wait_warp(dq_done, items & 1, abort_flag, P.err)) break;
-      ++items;
-      tc_fence_after();
-#pragma unroll
-      for (int cb = 0; cb < D / 2; cb += 32) {
-        const int col = half * (D / 2) + cb;
-        uint32_t ov[32];
-        tmem_ld32<0>(tmem_base + lane_off + C::kColDQ + col, ov);
-        tmem_wait_ld();
-        store_row32(P.dq + row * D + col, ov, P.scale);
-      }
-      tc_fence_before();
-      mbar_arrive(acc_free);
-    }
-  } else if (warp == 8) {
-    // ----------------------------------------------------------------- TMA --
-    uint32_t kv_idx = 0, items = 0;
-    bool ok = true;
-    for (int round = 0; ok; ++round) {
-      const int w = snake_item(round, cta, grid);
-      if (w >= P.n_items) break;
-      int qt, bh;
-      decode_item(P, w, true, qt, bh);
-      const int rowbase = bh * S;
-      if (items > 0 && !mbar_wait_warp(q_empty, (items - 1) & 1, abort_flag, P.err)) break;
-      if (lane == 0) {
-        mbar_expect_tx(q_full, 2 * C::kTileBytes);
-#pragma unroll
-        for (int sb = 0; sb < D / 64; ++sb) {
-          tma_load_2d(sQ + sb * C::kSubBytes, &tmQ, q_full, sb * 64, rowbase + qt * 128);
-          tma_load_2d(sdO + sb * C::kSubBytes, &tmdO, q_full, sb * 64, rowbase + qt * 128);
-        }
-      }
-      __syncwarp();
-      ++items;
-      KIter ki;
-      ki.init(P, qt);
-      int kt, dg;
-      while (ki.next(P, kt, dg)) {
-        for (int which = 0; which < 2; ++which) {
-          const int s = kv_idx % C::kStages;
-          if (kv_idx >= (uint32_t)C::kStages &&
-              !mbar_wait_warp(&kv_empty[s], ((kv_idx / C::kStages) - 1) & 1, abort_flag, P.err)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            mbar_expect_tx(&kv_full[s], C::kTileBytes);
-            const CUtensorMap* map = which ? &tmV : &tmK;
-#pragma unroll
-            for (int sb = 0; sb < D / 64; ++sb)
-              tma_load_2d(sKV + s * C::kTileBytes + sb * C::kSubBytes, map, &kv_full[s], sb * 64,
-                          rowbase + kt * 128);
-          }
-          __syncwarp();
-          ++kv_idx;
-        }
-        if (!ok) break;
-      }
-    }
-    if (*abort_flag) {
-      const unsigned long long t0 = globaltimer();
-      if (items > 0)
-        while (!mbar_try_wait(q_full, (items - 1) & 1) && globaltimer() - t0 < kWaitLimitNs) {
-        }
-      const uint32_t first = kv_idx > (uint32_t)C::kStages ? kv_idx - C::kStages : 0;
-      for (uint32_t i = first; i < kv_idx; ++i)
-        while (!mbar_try_wait(&kv_full[i % C::kStages], (i / C::kStages) & 1) &&
-               globaltimer() - t0 < kWaitLimitNs) {
-        }
-    }
-  } else {
-    // ----------------------------------------------------------------- MMA --
-    // Per K/V tile j: S(j+1) is issued before waiting for the elementwise work
-    // of tile j (two S buffers), then dQ += dS(j) K_j and dP(j+1).
-    const uint32_t tDP = tmem_base + C::kColDP, tDQ = tmem_base + C::kColDQ;
-    const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), aKV = smem_u32(sKV);
-    uint32_t kv_idx = 0, j_cnt = 0, items = 0;
-    bool ok = true;
-    auto issue_s = [&](uint32_t sbuf, uint32_t slotK) {
-      const uint32_t tS = tmem_base + (sbuf ? C::kColS1 : C::kColS0);
-      const uint32_t kb = aKV + slotK * C::kTileBytes;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tS, smem_desc_sw128(aQ + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-               C::kIdescS, kk > 0 ? 1u : 0u);
-      }
-    };
-    auto issue_dp = [&](uint32_t slotV) {
-      const uint32_t vb = aKV + slotV * C::kTileBytes;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tDP, smem_desc_sw128(adO + off, 16, 1024), smem_desc_sw128(vb + off, 16, 1024),
-               C::kIdescS, kk > 0 ? 1u : 0u);
-      }
-    };
-    for (int round = 0; ok; ++round) {
-      const int w = snake_item(round, cta, grid);
-      if (w >= P.n_items) break;
-      int qt, bh;
-      decode_item(P, w, true, qt, bh);
-      if (!mbar_wait_warp(q_full, items & 1, abort_flag, P.err)) break;
-      tc_fence_after();
-      KIter ki;
-      ki.init(P, qt);
-      int kt, dg;
-      // prologue: S(0), dP(0)
-      if (!ki.next(P, kt, dg)) break;  // unreachable: a q tile always sees its own block
-      uint32_t sK = kv_idx % C::kStages, phK = (kv_idx / C::kStages) & 1;
-      uint32_t sV = (kv_idx + 1) % C::kStages, phV = ((kv_idx + 1) / C::kStages) & 1;
-      kv_idx += 2;
-      if (!mbar_wait_warp(&kv_full[sK], phK, abort_flag, P.err)) { ok = false; break; }
-      tc_fence_after();
-      if (lane == 0) {
-        issue_s(j_cnt & 1, sK);
-        tc_commit(&s_ready[j_cnt & 1]);
-      }
-      __syncwarp();
-      if (!mbar_wait_warp(&kv_full[sV], phV, abort_flag, P.err)) { ok = false; break; }
-      tc_fence_after();
-      if (lane == 0) {
-        issue_dp(sV);
-        tc_commit(dp_ready);
-        tc_commit(&kv_empty[sV]);
-      }
-      __syncwarp();
-      bool first = true;
-      while (true) {
-        // S(j+1) into the other buffer, overlapping the elementwise work of j
-        const bool more = ki.next(P, kt, dg);
-        uint32_t sK2 = 0, sV2 = 0, phV2 = 0;
-        if (more) {
-          sK2 = kv_idx % C::kStages;
-          const uint32_t phK2 = (kv_idx / C::kStages) & 1;
-          sV2 = (kv_idx + 1) % C::kStages;
-          phV2 = ((kv_idx + 1) / C::kStages) & 1;
-          kv_idx += 2;
-          if (!mbar_wait_warp(&kv_full[sK2], phK2, abort_flag, P.err)) { ok = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
-            issue_s((j_cnt + 1) & 1, sK2);
-            tc_commit(&s_ready[(j_cnt + 1) & 1]);
-          }
-          __syncwarp();
-        }
-        if (!mbar_wait_warp(p_ready, j_cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        if (first && items > 0 && !mbar_wait_warp(acc_free, (items - 1) & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          // dQ += dS(j) K_j: A = dS packed in the S buffer, B = K_j MN-major over d
-          const uint32_t tS = tmem_base + ((j_cnt & 1) ? C::kColS1 : C::kColS0);
-          const uint32_t kb = aKV + sK * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDQ, tS + packed_kstep(kk), smem_desc_sw128(kb + kk * 2048, C::kSubBytes, 1024),
-                   C::kIdescDQ, (first && kk == 0) ? 0u : 1u);
-          tc_commit(&kv_empty[sK]);
-        }
-        __syncwarp();
-        first = false;
-        ++j_cnt;
-        if (!more) break;
-        if (!mbar_wait_warp(&kv_full[sV2], phV2, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
-          issue_dp(sV2);
-          tc_commit(dp_ready);
-          tc_commit(&kv_empty[sV2]);
-        }
-        __syncwarp();
-        sK = sK2;
-      }
-      if (!ok) break;
-      if (lane == 0) {
-        tc_commit(q_empty);  // every S / dP of this Q tile has been issued
-        tc_commit(dq_done);
       }
       __syncwarp();
       ++items;
@@ -842,16 +446,6 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   }
 }
 
-template <typename Cfg, typename Kern>
-bool set_smem(Kern kern, bool& done) {
-  if (done) return true;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
-      cudaSuccess)
-    return false;
-  done = true;
-  return true;
-}
-
 template <int D>
 int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v, const void* o,
                 const float* lse, const void* dout, void* dq, void* dk, void* dv, float* ws_delta,
@@ -879,14 +473,19 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.scale = sh.scale;
   P.lse2 = ws_lse2;
   P.delta = ws_delta;
+  P.q = static_cast<const __nv_bfloat16*>(q);
+  P.dout = static_cast<const __nv_bfloat16*>(dout);
   P.dq = static_cast<__nv_bfloat16*>(dq);
   P.dk = static_cast<__nv_bfloat16*>(dk);
   P.dv = static_cast<__nv_bfloat16*>(dv);
   P.err = err;
-  static bool attr_dkdv[2] = {false, false}, attr_dq[2] = {false, false};
-  if (!set_smem<DkdvCfg<D>>(tc_dkdv_kernel<D>, attr_dkdv[D == 128]) ||
-      !set_smem<DqCfg<D>>(tc_dq_kernel<D>, attr_dq[D == 128]))
-    return -1;
+  static bool attr[2] = {false, false};
+  if (!attr[D == 128]) {
+    if (cudaFuncSetAttribute(tc_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DkdvCfg<D>::kSmemBytes) != cudaSuccess)
+      return -1;
+    attr[D == 128] = true;
+  }
   int dev = 0;
   cudaGetDevice(&dev);
   int grid = num_sms(dev);
@@ -895,14 +494,12 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   tc_dkdv_kernel<D><<<grid, 320, DkdvCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
   prof_end(kKTcDkdv, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
-  prof_begin(kKTcDq, stream);
-  tc_dq_kernel<D><<<grid, 320, DqCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
-  prof_end(kKTcDq, stream);
-  if (cudaGetLastError() != cudaSuccess) return -1;
+  if (launch_tc_dq<D>(P, mq, mk, mv, mdo, grid, stream) < 0) return -1;
   return 3;
 }
 
 }  // namespace
+}  // namespace bwd
 
 bool tc_bwd_supported(const AttnShape& sh) {
   if (!sh.bf16) return false;
@@ -916,8 +513,8 @@ int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void*
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
                   void* dv, float* ws_delta, float* ws_lse2, unsigned* err, cudaStream_t stream) {
   if (sh.D == 64)
-    return launch_impl<64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
-  return launch_impl<128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
+    return bwd::launch_impl<64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
+  return bwd::launch_impl<128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
 }
 
 }  // namespace cpattn
