@@ -269,6 +269,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// Descriptor of the same layout at a byte offset (a multiple of 16) from `d`.
+// The MMA thread builds one descriptor per operand tile and derives each
+// k-step from it with one add (the offsets are constants once the k-loop is
+// unrolled), which keeps its issue rate at the tensor core's pace; the add
+// never carries out of the 14-bit address field because every address stays
+// inside the CTA's shared memory.
+__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) {
+  return d + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 // a_mn / b_mn: 1 when that operand is MN-major (contiguous along M / N).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {

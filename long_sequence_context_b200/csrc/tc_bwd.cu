@@ -309,22 +309,32 @@ __global__ void __launch_bounds__(320, 1)
     auto q_addr = [&](uint32_t cnt) {
       return smem_u32(smem + C::kOffQ + (2 * (cnt % C::kStages)) * C::kTileBytes);
     };
+    // One descriptor per operand tile; k-steps are constant offsets from it.
+    const uint64_t dK0 = smem_desc_sw128(aK, 16, 1024), dV0 = smem_desc_sw128(aV, 16, 1024);
     // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
     auto issue_st = [&](uint32_t aQ) {
+      const uint64_t dq = smem_desc_sw128(aQ, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tS, smem_desc_sw128(aK + off, 16, 1024), smem_desc_sw128(aQ + off, 16, 1024),
-               C::kIdescST, kk > 0 ? 1u : 0u);
+        mma_ss(tS, desc_at(dK0, off), desc_at(dq, off), C::kIdescST, kk > 0 ? 1u : 0u);
       }
     };
     auto issue_dpt = [&](uint32_t adO) {
+      const uint64_t ddo = smem_desc_sw128(adO, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tDP, smem_desc_sw128(aV + off, 16, 1024), smem_desc_sw128(adO + off, 16, 1024),
-               C::kIdescST, kk > 0 ? 1u : 0u);
+        mma_ss(tDP, desc_at(dV0, off), desc_at(ddo, off), C::kIdescST, kk > 0 ? 1u : 0u);
       }
+    };
+    // acc += (packed TMEM operand) x (B MN-major over d)
+    auto issue_acc = [&](uint32_t t_acc, uint32_t t_a, uint32_t aB, bool first) {
+      const uint64_t db = smem_desc_sw128(aB, C::kSubBytes, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(t_acc, t_a + packed_kstep(kk), desc_at(db, kk * 2048), C::kIdescAcc,
+               (first && kk == 0) ? 0u : 1u);
     };
     // Per q tile t the order is dV(t), S^T(t+1), dK(t), dP^T(t+1): dV(t) and
     // S^T(t+1) run under the dS phase of t, dK(t) and dP^T(t+1) under the
@@ -360,12 +370,7 @@ __global__ void __launch_bounds__(320, 1)
           break;
         }
         tc_fence_after();
-        if (lane == 0) {  // dV += P^T dO (A packed in TMEM, B MN-major over d)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDV, tS + packed_kstep(kk), smem_desc_sw128(adO + kk * 2048, C::kSubBytes, 1024),
-                   C::kIdescAcc, (t == 0 && kk == 0) ? 0u : 1u);
-        }
+        if (lane == 0) issue_acc(tDV, tS, adO, t == 0);  // dV += P^T dO
         __syncwarp();
         if (t + 1 < n) {
           if (!mbar_wait_warp(&q_full[(cnt + 1) % C::kStages], ((cnt + 1) / C::kStages) & 1, abort_flag,
@@ -382,11 +387,8 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!mbar_wait_warp(pb_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
         tc_fence_after();
-        if (lane == 0) {  // dK += dS^T Q
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDK, tDP + packed_kstep(kk), smem_desc_sw128(aQ + kk * 2048, C::kSubBytes, 1024),
-                   C::kIdescAcc, (t == 0 && kk == 0) ? 0u : 1u);
+        if (lane == 0) {
+          issue_acc(tDK, tDP, aQ, t == 0);  // dK += dS^T Q
           tc_commit(&q_empty[cnt % C::kStages]);
           if (t + 1 < n) {
             issue_dpt(q_addr(cnt + 1) + C::kTileBytes);

@@ -259,22 +259,23 @@ __global__ void __launch_bounds__(320, 1)
     // slot of K / V tile t of the current item: kv_base + 2t (+1 for V)
     auto slot_of = [&](uint32_t idx) { return idx % C::kStages; };
     auto phase_of = [&](uint32_t idx) { return (idx / C::kStages) & 1; };
+    // One descriptor per operand tile; k-steps are constant offsets from it.
+    const uint64_t dQ0 = smem_desc_sw128(aQ, 16, 1024), ddO0 = smem_desc_sw128(adO, 16, 1024);
     auto issue_s = [&](int buf, uint32_t slotK) {
-      const uint32_t kb = aKV + slotK * C::kTileBytes;
+      const uint64_t dk = smem_desc_sw128(aKV + slotK * C::kTileBytes, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tmem_base + C::col_s(buf), smem_desc_sw128(aQ + off, 16, 1024),
-               smem_desc_sw128(kb + off, 16, 1024), C::kIdescS, kk > 0 ? 1u : 0u);
+        mma_ss(tmem_base + C::col_s(buf), desc_at(dQ0, off), desc_at(dk, off), C::kIdescS,
+               kk > 0 ? 1u : 0u);
       }
     };
     auto issue_dp = [&](uint32_t slotV) {
-      const uint32_t vb = aKV + slotV * C::kTileBytes;
+      const uint64_t dv = smem_desc_sw128(aKV + slotV * C::kTileBytes, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tDP, smem_desc_sw128(adO + off, 16, 1024), smem_desc_sw128(vb + off, 16, 1024),
-               C::kIdescS, kk > 0 ? 1u : 0u);
+        mma_ss(tDP, desc_at(ddO0, off), desc_at(dv, off), C::kIdescS, kk > 0 ? 1u : 0u);
       }
     };
     for (int round = 0; ok; ++round) {
@@ -339,11 +340,12 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (lane == 0) {  // dQ += dS_t K_t
           const uint32_t tDS = tmem_base + C::col_s(j_cnt & 1);
-          const uint32_t kb = aKV + slot_of(base + 2 * t) * C::kTileBytes;
+          const uint64_t dk = smem_desc_sw128(aKV + slot_of(base + 2 * t) * C::kTileBytes,
+                                              C::kSubBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDQ, tDS + packed_kstep(kk), smem_desc_sw128(kb + kk * 2048, C::kSubBytes, 1024),
-                   C::kIdescDQ, (t == 0 && kk == 0) ? 0u : 1u);
+            mma_ts(tDQ, tDS + packed_kstep(kk), desc_at(dk, kk * 2048), C::kIdescDQ,
+                   (t == 0 && kk == 0) ? 0u : 1u);
           tc_commit(&kv_empty[slot_of(base + 2 * t)]);
         }
         __syncwarp();

@@ -401,6 +401,24 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO[2] = {tmem_base + 256, tmem_base + 384};
     const uint32_t aQ[2] = {smem_u32(sQ[0]), smem_u32(sQ[1])};
     const uint32_t aKV = smem_u32(sKV);
+    // one descriptor per operand tile; k-steps are constant offsets from it
+    const uint64_t dQd[2] = {smem_desc_sw128(aQ[0], 16, 1024), smem_desc_sw128(aQ[1], 16, 1024)};
+    // O += P V: A = P (bf16, two per TMEM column), B = V (MN-major over d)
+    auto issue_pv = [&](uint32_t t_o, uint32_t t_p, uint32_t slot_v, bool first) {
+      const uint64_t dv = smem_desc_sw128(aKV + slot_v * C::kTileBytes, C::kSubBytes, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(t_o, t_p + kk * 8, desc_at(dv, kk * 2048), C::kIdescPV, (first && kk == 0) ? 0u : 1u);
+    };
+    // S = Q K^T: both operands K-major
+    auto issue_qk = [&](uint32_t t_s, uint64_t dq, uint32_t slot_k) {
+      const uint64_t dk = smem_desc_sw128(aKV + slot_k * C::kTileBytes, 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+        mma_ss(t_s, desc_at(dq, off), desc_at(dk, off), C::kIdescQK, kk > 0 ? 1u : 0u);
+      }
+    };
     uint32_t kv_idx = 0, p_cnt = 0, n_items = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
@@ -430,20 +448,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         tc_fence_after();
         if (lane == 0) {
-          if (has_prev) {
-            const uint32_t vb = aKV + prev_sV * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tO[0], tS[0] + kk * 8, smem_desc_sw128(vb + kk * 2048, C::kSubBytes, 1024),
-                     C::kIdescPV, (prev_first && kk == 0) ? 0u : 1u);
-          }
-          const uint32_t kb = aKV + sK * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-            mma_ss(tS[0], smem_desc_sw128(aQ[0] + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                   C::kIdescQK, kk > 0 ? 1u : 0u);
-          }
+          if (has_prev) issue_pv(tO[0], tS[0], prev_sV, prev_first);
+          issue_qk(tS[0], dQd[0], sK);
           tc_commit(&s_ready[0]);
         }
         __syncwarp();
@@ -454,20 +460,10 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (lane == 0) {
           if (has_prev) {
-            const uint32_t vb = aKV + prev_sV * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ts(tO[1], tS[1] + kk * 8, smem_desc_sw128(vb + kk * 2048, C::kSubBytes, 1024),
-                     C::kIdescPV, (prev_first && kk == 0) ? 0u : 1u);
+            issue_pv(tO[1], tS[1], prev_sV, prev_first);
             tc_commit(&kv_empty[prev_sV]);
           }
-          const uint32_t kb = aKV + sK * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-            mma_ss(tS[1], smem_desc_sw128(aQ[1] + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                   C::kIdescQK, kk > 0 ? 1u : 0u);
-          }
+          issue_qk(tS[1], dQd[1], sK);
           tc_commit(&s_ready[1]);
           tc_commit(&kv_empty[sK]);
         }
@@ -485,11 +481,7 @@ __global__ void __launch_bounds__(384, 1)
           !mbar_wait_warp(&p_ready[0], p_cnt & 1, abort_flag, P.err)) break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vb = aKV + prev_sV * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tO[0], tS[0] + kk * 8, smem_desc_sw128(vb + kk * 2048, C::kSubBytes, 1024),
-                 C::kIdescPV, (prev_first && kk == 0) ? 0u : 1u);
+        issue_pv(tO[0], tS[0], prev_sV, prev_first);
         tc_commit(&o_ready[0]);
       }
       __syncwarp();
@@ -497,11 +489,7 @@ __global__ void __launch_bounds__(384, 1)
       ++p_cnt;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vb = aKV + prev_sV * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tO[1], tS[1] + kk * 8, smem_desc_sw128(vb + kk * 2048, C::kSubBytes, 1024),
-                 C::kIdescPV, (prev_first && kk == 0) ? 0u : 1u);
+        issue_pv(tO[1], tS[1], prev_sV, prev_first);
         tc_commit(&o_ready[1]);
         tc_commit(&kv_empty[prev_sV]);
       }
