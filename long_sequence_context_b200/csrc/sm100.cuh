@@ -84,6 +84,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// A barrier test whose result is needed only later.  The thread that issues
+// MMAs tests the barrier of its next group between two MMAs of the current
+// one: the test's latency then overlaps queued tensor work instead of leaving
+// the tensor pipe idle between groups (the pipe queues very few MMAs ahead of
+// the issuing thread).
+struct Probe {
+  uint64_t* bar = nullptr;  // nullptr: nothing to test
+  uint32_t parity = 0;
+  bool done = true;
+  __device__ __forceinline__ void set(uint64_t* b, uint32_t p) {
+    bar = b;
+    parity = p;
+    done = false;
+  }
+  __device__ __forceinline__ void test() {
+    if (bar != nullptr && !done) done = mbar_try_wait(bar, parity);
+  }
+  // complete the wait if the early test did not see the phase finished
+  __device__ __forceinline__ bool finish(volatile int* abort_flag, unsigned* err) {
+    const bool r = done || mbar_wait(bar, parity, abort_flag, err);
+    bar = nullptr;
+    done = true;
+    return r;
+  }
+};
+
 // The same wait taken by a whole warp: the outcome is made warp-uniform, so a
 // warp never splits around the warp-collective (.sync.aligned) tcgen05
 // instructions that follow a wait.

@@ -301,93 +301,91 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ----------------------------------------------------------------- MMA --
-    const uint32_t tS = tmem_base + C::kColS, tDP = tmem_base + C::kColDP;
-    const uint32_t tDV = tmem_base + C::kColDV, tDK = tmem_base + C::kColDK;
-    const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-    uint32_t items = 0, q_cnt = 0;
-    bool ok = true;
-    auto q_addr = [&](uint32_t cnt) {
-      return smem_u32(smem + C::kOffQ + (2 * (cnt % C::kStages)) * C::kTileBytes);
-    };
-    // One descriptor per operand tile; k-steps are constant offsets from it.
-    const uint64_t dK0 = smem_desc_sw128(aK, 16, 1024), dV0 = smem_desc_sw128(aV, 16, 1024);
-    // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
-    auto issue_st = [&](uint32_t aQ) {
-      const uint64_t dq = smem_desc_sw128(aQ, 16, 1024);
+    // One thread issues every MMA (the other lanes wait at the end).  The
+    // tensor pipe queues very few MMAs ahead of it, so a barrier wait between
+    // two MMA groups leaves the pipe idle; the wait for the next q tile's
+    // operands is therefore tested (Probe) between the MMAs of dV.
+    if (lane == 0) {
+      const uint32_t tS = tmem_base + C::kColS, tDP = tmem_base + C::kColDP;
+      const uint32_t tDV = tmem_base + C::kColDV, tDK = tmem_base + C::kColDK;
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+      uint32_t items = 0, q_cnt = 0;
+      bool ok = true;
+      Probe pr;
+      auto q_addr = [&](uint32_t cnt) {
+        return smem_u32(smem + C::kOffQ + (2 * (cnt % C::kStages)) * C::kTileBytes);
+      };
+      // One descriptor per operand tile; k-steps are constant offsets from it.
+      const uint64_t dK0 = smem_desc_sw128(aK, 16, 1024), dV0 = smem_desc_sw128(aV, 16, 1024);
+      // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+      auto issue_st = [&](uint32_t aQ) {
+        const uint64_t dq = smem_desc_sw128(aQ, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tS, desc_at(dK0, off), desc_at(dq, off), C::kIdescST, kk > 0 ? 1u : 0u);
-      }
-    };
-    auto issue_dpt = [&](uint32_t adO) {
-      const uint64_t ddo = smem_desc_sw128(adO, 16, 1024);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+          mma_ss(tS, desc_at(dK0, off), desc_at(dq, off), C::kIdescST, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_dpt = [&](uint32_t adO) {
+        const uint64_t ddo = smem_desc_sw128(adO, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(tDP, desc_at(dV0, off), desc_at(ddo, off), C::kIdescST, kk > 0 ? 1u : 0u);
-      }
-    };
-    // acc += (packed TMEM operand) x (B MN-major over d)
-    auto issue_acc = [&](uint32_t t_acc, uint32_t t_a, uint32_t aB, bool first) {
-      const uint64_t db = smem_desc_sw128(aB, C::kSubBytes, 1024);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+          mma_ss(tDP, desc_at(dV0, off), desc_at(ddo, off), C::kIdescST, kk > 0 ? 1u : 0u);
+        }
+      };
+      // acc += (packed TMEM operand) x (B MN-major over d); tests the probe
+      // between k-steps
+      auto issue_acc = [&](uint32_t t_acc, uint32_t t_a, uint32_t aB, bool first) {
+        const uint64_t db = smem_desc_sw128(aB, C::kSubBytes, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts(t_acc, t_a + packed_kstep(kk), desc_at(db, kk * 2048), C::kIdescAcc,
-               (first && kk == 0) ? 0u : 1u);
-    };
-    // Per q tile t the order is dV(t), S^T(t+1), dK(t), dP^T(t+1): dV(t) and
-    // S^T(t+1) run under the dS phase of t, dK(t) and dP^T(t+1) under the
-    // exponential phase of t+1.
-    for (int round = 0; ok; ++round) {
-      const int w = snake_item(round, cta, grid);
-      if (w >= P.n_items) break;
-      int jt, bh;
-      decode_item(P, w, false, jt, bh);
-      QIter qi;
-      qi.init(P, jt);
-      int n = 0, qt, dg;
-      while (qi.next(P, qt, dg)) ++n;
-      const uint32_t base = q_cnt;
-      q_cnt += n;
-      if (!mbar_wait_warp(kv_full, items & 1, abort_flag, P.err) ||
-          !mbar_wait_warp(&q_full[base % C::kStages], (base / C::kStages) & 1, abort_flag, P.err))
-        break;
-      tc_fence_after();
-      if (lane == 0) {
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_ts(t_acc, t_a + packed_kstep(kk), desc_at(db, kk * 2048), C::kIdescAcc,
+                 (first && kk == 0) ? 0u : 1u);
+          if (kk == 2 || kk == 6) pr.test();
+        }
+      };
+      // Per q tile t the order is dV(t), S^T(t+1), dK(t), dP^T(t+1): dV(t) and
+      // S^T(t+1) run under the dS phase of t, dK(t) and dP^T(t+1) under the
+      // exponential phase of t+1.
+      for (int round = 0; ok; ++round) {
+        const int w = snake_item(round, cta, grid);
+        if (w >= P.n_items) break;
+        int jt, bh;
+        decode_item(P, w, false, jt, bh);
+        QIter qi;
+        qi.init(P, jt);
+        int n = 0, qt, dg;
+        while (qi.next(P, qt, dg)) ++n;
+        const uint32_t base = q_cnt;
+        q_cnt += n;
+        if (!mbar_wait(kv_full, items & 1, abort_flag, P.err) ||
+            !mbar_wait(&q_full[base % C::kStages], (base / C::kStages) & 1, abort_flag, P.err))
+          break;
+        tc_fence_after();
         issue_st(q_addr(base));
         tc_commit(s_ready);
         issue_dpt(q_addr(base) + C::kTileBytes);
         tc_commit(dp_ready);
-      }
-      __syncwarp();
-      for (int t = 0; t < n; ++t) {
-        const uint32_t cnt = base + t;
-        const uint32_t aQ = q_addr(cnt), adO = aQ + C::kTileBytes;
-        if (!mbar_wait_warp(pa_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        if (t == 0 && items > 0 && !mbar_wait_warp(acc_free, (items - 1) & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) issue_acc(tDV, tS, adO, t == 0);  // dV += P^T dO
-        __syncwarp();
-        if (t + 1 < n) {
-          if (!mbar_wait_warp(&q_full[(cnt + 1) % C::kStages], ((cnt + 1) / C::kStages) & 1, abort_flag,
-                              P.err)) {
+        for (int t = 0; t < n; ++t) {
+          const uint32_t cnt = base + t;
+          const uint32_t aQ = q_addr(cnt), adO = aQ + C::kTileBytes;
+          if (!mbar_wait(pa_ready, cnt & 1, abort_flag, P.err) ||
+              (t == 0 && items > 0 && !mbar_wait(acc_free, (items - 1) & 1, abort_flag, P.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (lane == 0) {
+          if (t + 1 < n) pr.set(&q_full[(cnt + 1) % C::kStages], ((cnt + 1) / C::kStages) & 1);
+          issue_acc(tDV, tS, adO, t == 0);  // dV += P^T dO
+          if (t + 1 < n) {
+            if (!pr.finish(abort_flag, P.err)) { ok = false; break; }
+            tc_fence_after();
             issue_st(q_addr(cnt + 1));
             tc_commit(s_ready);
           }
-          __syncwarp();
-        }
-        if (!mbar_wait_warp(pb_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
+          if (!mbar_wait(pb_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
+          tc_fence_after();
           issue_acc(tDK, tDP, aQ, t == 0);  // dK += dS^T Q
           tc_commit(&q_empty[cnt % C::kStages]);
           if (t + 1 < n) {
@@ -395,21 +393,17 @@ __global__ void __launch_bounds__(320, 1)
             tc_commit(dp_ready);
           }
         }
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (lane == 0) {
+        if (!ok) break;
         tc_commit(kv_empty);
         tc_commit(kv_done);
+        ++items;
       }
-      __syncwarp();
-      ++items;
+      tc_commit(drain);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
     }
-    if (lane == 0) tc_commit(drain);
     __syncwarp();
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
-    }
   }
 
   __syncthreads();
