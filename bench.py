@@ -30,6 +30,47 @@ DEFAULT_WORKLOAD = "causal_b1h32s32768d128_cp8_bf16"
 METRIC = "causal ring-attn TFLOP/s fwd & fwd+bwd on 1 B200; % of BF16 tensor peak"
 
 
+# DRAM traffic of the dominant kernel, read from a committed ncu summary.  The
+# summary records a digest of the kernel's sources at capture time; when the
+# sources have changed since, the figure no longer describes the kernel and
+# traffic is reported as null.
+TRAFFIC_FILES = {
+    ("tc_dkdv", "causal_b1h32s32768d128_cp8_bf16"):
+        os.path.join(ROOT, "profiles", "traffic_tc_dkdv_causal_b1h32s32768d128_cp8.txt"),
+}
+KERNEL_SOURCES = {
+    "tc_dkdv": ["tc_bwd.cu", "bwd_common.cuh", "kernels.h", "sm100.cuh", "tmap.h", "ring.cuh"],
+}
+
+
+def kernel_source_digest(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "long_sequence_context_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel, workload):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch, or None."""
+    path = TRAFFIC_FILES.get((kernel, workload))
+    if path is None or not os.path.exists(path):
+        return None
+    rec = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                rec[k.strip()] = v.strip()
+    if rec.get("source_sha256") != kernel_source_digest(kernel):
+        return None
+    try:
+        return int(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -289,7 +330,7 @@ def run_gpu(args, w):
         roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
                 "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "unit": "TFLOP/s",
                 "frac": ach / peak, "frac_of_burst_peak": ach / peaks["bf16_tflops"],
-                "traffic": None}
+                "traffic": recorded_traffic(dom, w.name), "traffic_unit": "bytes per launch"}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
