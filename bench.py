@@ -60,7 +60,7 @@ def recorded_traffic(kernel, workload):
     rec = {}
     with open(path) as f:
         for line in f:
-            if ":" in line:
+            if ":" in line and not line.lstrip().startswith("#"):
                 k, v = line.split(":", 1)
                 rec[k.strip()] = v.strip()
     if rec.get("source_sha256") != kernel_source_digest(kernel):
