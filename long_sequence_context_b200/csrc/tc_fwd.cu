@@ -248,9 +248,17 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < 128; ++c)
             if (c > lim) r[c] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(r[0]);
+        // row maximum as 8 independent chains (a single chain of 127 dependent
+        // max operations would put its full latency on every tile)
+        float mp[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+        for (int i = 0; i < 8; ++i) mp[i] = __uint_as_float(r[i]);
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mp[i] = fmaxf(mp[i], __uint_as_float(r[c + i]));
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
         const float m_tile = mx * P.sl2;
         float m_new = m;
         if (m_tile > m + kRescaleThreshold || m == -INFINITY) m_new = fmaxf(m, m_tile);
@@ -262,15 +270,15 @@ __global__ void __launch_bounds__(384, 1)
         if (j > 0 && __any_sync(0xffffffffu, grow)) rescale_rows<D>(tO, f);
         m = m_new;
         const float base = (m == -INFINITY) ? 0.f : m;
-        float lsum = 0.f;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
           const float p0 = ex2(fmaf(__uint_as_float(r[c]), P.sl2, -base));
           const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), P.sl2, -base));
-          lsum += p0 + p1;
+          ls[(c >> 1) & 3] += p0 + p1;
           r[c >> 1] = pack_bf16x2(p0, p1);  // r[c/2] was read at or before this step
         }
-        l += lsum;
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tmem_st32<0>(tS + 0, r);
         tmem_st32<32>(tS + 32, r);
         tmem_wait_st();
