@@ -398,6 +398,91 @@ def run_gpu(args, w):
         dist.destroy_process_group()
 
 
+LAYER_METRIC = "attention layer (projections + ring attention) TFLOP/s fwd+bwd on 1 B200"
+
+
+def run_layer(args, w):
+    """The attention layer around the ring attention, forward + backward per
+    step: E = H * D of the workload, B, S, cp_size, causal as in it.  Separate
+    from the headline line; prints its own JSON line."""
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    from long_sequence_context_b200 import cpattn as cp
+    from long_sequence_context_b200.inputs import flops_layer, make_layer_inputs
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    B, S, H, D = w.B, w.S, w.H, w.D
+    E = H * D
+    x, w_qkv, b_qkv, w_o, b_o, dy = (t.to(dev) for t in make_layer_inputs(B, S, E, seed=w.seed))
+    ws = torch.empty(cp.layer_workspace_bytes(B, S, E, H), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        _, saved = cp.layer_fwd(x, w_qkv, b_qkv, w_o, b_o, H, w.cp_size, w.causal, w.scale, workspace=ws)
+        cp.layer_bwd(x, w_qkv, w_o, saved, dy, H, w.cp_size, w.causal, w.scale, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    if cp.sync_status() != cp.OK:
+        raise RuntimeError("layer warm-up failed")
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    n0 = cp.launch_count()
+    cp.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    cp.profile(False)
+    launches = cp.launch_count() - n0
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    clk = clocks.stop()
+    if cp.sync_status() != cp.OK:
+        raise RuntimeError("layer timed region failed")
+    f_fwd, f_bwd = flops_layer(B, S, E, H, w.causal)
+    ms_step = ms_total / args.steps
+    per_kernel = {}
+    for kind, name in cp.KERNEL_KINDS.items():
+        ms, n = cp.profile_read(kind)
+        if n:
+            per_kernel[name] = {"ms_total": ms, "launches": n, "ms_avg": ms / n}
+    own_ms = sum(v["ms_total"] for v in per_kernel.values()) / args.steps
+    # head reshapes per step: q|k|v split, O merge (fwd and bwd), dO split, dQ|dK|dV merge:
+    # each reads and writes its tensor once: (3 + 1 + 1 + 1 + 3) * B*S*E bf16 elements, x2
+    heads_bytes = 9 * B * S * E * 2 * 2
+    hk = per_kernel.get("layer_heads")
+    heads_roof = None
+    if hk:
+        ach = heads_bytes / (hk["ms_total"] / args.steps * 1e-3) / 1e9
+        heads_roof = {"bound": "hbm", "kernel": "layer_heads", "achieved": ach, "peak": peaks["hbm_gbs"],
+                      "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    if rank == 0:
+        line = {
+            "metric": LAYER_METRIC, "value": (f_fwd + f_bwd) * world / (ms_step * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (nn.Linear-range random weights)",
+            "config": {"workload": f"layer_{w.name}", "B": B, "S": S, "E": E, "H": H, "D": D,
+                       "cp_size": w.cp_size, "causal": w.causal},
+            "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd},
+            "per_kernel_ms": per_kernel,
+            "cublaslt_gemm_ms_per_step": ms_step - own_ms,
+            "heads_roofline": heads_roof,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -408,6 +493,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fwd-only", action="store_true", help="time the forward alone (profiling)")
+    ap.add_argument("--layer", action="store_true",
+                    help="time the attention layer (projections + ring attention) instead")
     ap.add_argument("--shape", default=None,
                     help="B,H,S,D,cp_size,causal: a smaller case of the workload (profiling)")
     args = ap.parse_args()
@@ -422,6 +509,8 @@ def main():
                                 cp_size=N, causal=bool(c))
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.layer:
+        run_layer(args, w)
     else:
         run_gpu(args, w)
 

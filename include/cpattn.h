@@ -183,6 +183,47 @@ int cpattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* 
                        void* stream);
 
 /*
+ * The attention layer around the ring attention ("Configuring
+ * RingAttention+FlashAttention for CP", section 3 code): Q, K, V projections
+ * of width E (nn.Linear with bias), the [B,S,E] -> [B,H,S,D] head split, the
+ * ring attention (cpattn_fwd), the head merge and the output projection.
+ * bf16 only; D = E / H must be 64 or 128 and the attention's own
+ * preconditions apply to (B, H, S, D, cp_size, causal).
+ *   Layouts (row-major, caller-owned device memory, 16-byte aligned):
+ *     x, y, dy, dx           [B][S][E]
+ *     w_qkv, dw_qkv          [3E][E]   rows = the q, k and v projection weights
+ *                                      stacked (out features x in features)
+ *     b_qkv, db_qkv          [3E]
+ *     w_o, dw_o              [E][E];   b_o, db_o [E]
+ *     q, k, v, o             [B][H][S][D] (bf16), lse [B][H][S] (fp32): saved
+ *                                      by the forward for the backward
+ *   The projections run on cuBLASLt (bf16, fp32 accumulation, the bias added
+ *   in the GEMM epilogue) with the caller's workspace; the head reshapes and
+ *   the bias gradients are this library's kernels.
+ *   Workspace: cpattn_layer_workspace_bytes(B, S, E, H) bytes (0 for invalid
+ *   sizes), used by both calls; its contents need not survive between them.
+ *   Errors: CPATTN_ERR_SHAPE / ARG / ALIGN / WORKSPACE before anything is
+ *   enqueued; CPATTN_ERR_CUDA when a launch or a cuBLASLt call fails.
+ */
+size_t cpattn_layer_workspace_bytes(int B, int S, int E, int H);
+
+/* y = out_proj(merge_heads(attention(split_heads(x w_qkv^T + b_qkv)))) */
+int cpattn_layer_fwd(const void* x, const void* w_qkv, const void* b_qkv, const void* w_o,
+                     const void* b_o, void* y, void* q, void* k, void* v, void* o, float* lse,
+                     int B, int S, int E, int H, int cp_size, int causal, float scale,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Gradients of the layer for upstream gradient dy, from the forward's saved
+ * q, k, v, o, lse: dx, dw_qkv, db_qkv, dw_o, db_o (all overwritten).
+ */
+int cpattn_layer_bwd(const void* x, const void* w_qkv, const void* w_o, const void* q,
+                     const void* k, const void* v, const void* o, const float* lse,
+                     const void* dy, void* dx, void* dw_qkv, void* db_qkv, void* dw_o,
+                     void* db_o, int B, int S, int E, int H, int cp_size, int causal,
+                     float scale, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * cpattn_sync_status -- synchronises `stream`, then returns and clears the
  * device-side error word of the current device (CPATTN_OK, CPATTN_ERR_TIMEOUT)
  * or CPATTN_ERR_CUDA if the synchronisation itself failed.
@@ -216,7 +257,8 @@ long long cpattn_launch_count(void);
  *   since the last cpattn_profile(1); waits for those events.  Kernel kinds:
  *   0 tcgen05 forward, 1 CUDA-core forward, 2 merge, 3 finalize, 4 backward
  *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 dK/dV,
- *   8 tcgen05 dQ.
+ *   8 tcgen05 dQ, 9 layer head split / merge, 10 layer bias gradients (the
+ *   layer's cuBLASLt GEMMs are not this library's kernels and are not timed).
  */
 int cpattn_profile(int on);
 int cpattn_profile_read(int kernel_kind, double* total_ms, long long* launches);

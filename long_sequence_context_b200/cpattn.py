@@ -23,7 +23,8 @@ PLAN_FIELDS = 6
 EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpattn_finalize",
            "cpattn_bwd_workspace_bytes", "cpattn_bwd", "cpattn_sync_status",
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
-           "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc"]
+           "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc",
+           "cpattn_layer_workspace_bytes", "cpattn_layer_fwd", "cpattn_layer_bwd"]
 
 # size of the library's fixed scratch array behind bwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -58,6 +59,9 @@ def _load():
         "cpattn_bwd_noalloc": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp], i),
         "cpattn_profile": ([i], i),
         "cpattn_profile_read": ([i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], i),
+        "cpattn_layer_workspace_bytes": ([i, i, i, i], sz),
+        "cpattn_layer_fwd": ([vp] * 11 + [i] * 6 + [f, vp, sz, vp], i),
+        "cpattn_layer_bwd": ([vp] * 14 + [i] * 6 + [f, vp, sz, vp], i),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(L, name)
@@ -205,6 +209,69 @@ def bwd_noalloc(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=
     return dq, dk, dv
 
 
+def layer_workspace_bytes(B, S, E, H) -> int:
+    return int(lib.cpattn_layer_workspace_bytes(B, S, E, H))
+
+
+def _bf16(t, name, shape):
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bf16")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return _dev(t, name)
+
+
+def layer_fwd(x, w_qkv, b_qkv, w_o, b_o, num_heads: int, cp_size: int, causal: bool = True,
+              scale=None, workspace=None, stream=None):
+    """Attention layer forward (projections, head split, ring attention, head
+    merge, output projection).  Returns (y, saved) where saved = (q, k, v, o,
+    lse) feeds layer_bwd."""
+    B, S, E = x.shape
+    H = num_heads
+    D = E // H
+    scale = float(scale if scale is not None else D ** -0.5)
+    if workspace is None:
+        workspace = torch.empty(layer_workspace_bytes(B, S, E, H), dtype=torch.uint8, device=x.device)
+    y = torch.empty_like(x)
+    q, k, v, o = (torch.empty((B, H, S, D), dtype=x.dtype, device=x.device) for _ in range(4))
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=x.device)
+    st = lib.cpattn_layer_fwd(_bf16(x, "x", (B, S, E)), _bf16(w_qkv, "w_qkv", (3 * E, E)),
+                              _bf16(b_qkv, "b_qkv", (3 * E,)), _bf16(w_o, "w_o", (E, E)),
+                              _bf16(b_o, "b_o", (E,)), _dev(y, "y"), _dev(q, "q"), _dev(k, "k"),
+                              _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"), B, S, E, H, cp_size,
+                              int(causal), scale, ctypes.c_void_p(workspace.data_ptr()),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "cpattn_layer_fwd")
+    return y, (q, k, v, o, lse)
+
+
+def layer_bwd(x, w_qkv, w_o, saved, dy, num_heads: int, cp_size: int, causal: bool = True,
+              scale=None, workspace=None, stream=None):
+    """Attention layer backward: returns (dx, dw_qkv, db_qkv, dw_o, db_o)."""
+    B, S, E = x.shape
+    H = num_heads
+    D = E // H
+    scale = float(scale if scale is not None else D ** -0.5)
+    q, k, v, o, lse = saved
+    if workspace is None:
+        workspace = torch.empty(layer_workspace_bytes(B, S, E, H), dtype=torch.uint8, device=x.device)
+    dx = torch.empty_like(x)
+    dw_qkv = torch.empty_like(w_qkv)
+    db_qkv = torch.empty((3 * E,), dtype=x.dtype, device=x.device)
+    dw_o = torch.empty_like(w_o)
+    db_o = torch.empty((E,), dtype=x.dtype, device=x.device)
+    st = lib.cpattn_layer_bwd(_bf16(x, "x", (B, S, E)), _bf16(w_qkv, "w_qkv", (3 * E, E)),
+                              _bf16(w_o, "w_o", (E, E)), _bf16(q, "q", (B, H, S, D)),
+                              _bf16(k, "k", (B, H, S, D)), _bf16(v, "v", (B, H, S, D)),
+                              _bf16(o, "o", (B, H, S, D)), _dev(lse, "lse"), _bf16(dy, "dy", (B, S, E)),
+                              _dev(dx, "dx"), _dev(dw_qkv, "dw_qkv"), _dev(db_qkv, "db_qkv"),
+                              _dev(dw_o, "dw_o"), _dev(db_o, "db_o"), B, S, E, H, cp_size, int(causal),
+                              scale, ctypes.c_void_p(workspace.data_ptr()),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "cpattn_layer_bwd")
+    return dx, dw_qkv, db_qkv, dw_o, db_o
+
+
 def sync_status(stream=None) -> int:
     return int(lib.cpattn_sync_status(_stream(stream)))
 
@@ -230,7 +297,8 @@ def debug_stall(n: int) -> int:
 
 
 KERNEL_KINDS = {0: "tc_fwd", 1: "simt_fwd", 2: "merge", 3: "finalize", 4: "bwd_delta",
-                5: "simt_dkdv", 6: "simt_dq", 7: "tc_dkdv", 8: "tc_dq"}
+                5: "simt_dkdv", 6: "simt_dq", 7: "tc_dkdv", 8: "tc_dq", 9: "layer_heads",
+                10: "layer_colsum"}
 
 
 def profile(on: bool) -> int:

@@ -86,6 +86,20 @@ int check_shape(int B, int H, int S, int D, int cp_size, int causal, float scale
   return CPATTN_OK;
 }
 
+}  // namespace
+
+namespace cpattn {
+int check_attention_shape(int B, int H, int S, int D, int cp_size, int causal, float scale,
+                          int dtype) {
+  AttnShape sh;
+  return check_shape(B, H, S, D, cp_size, causal, scale, dtype, &sh);
+}
+
+void add_launches(int n) { g_launches += n; }
+}  // namespace cpattn
+
+namespace {
+
 bool use_tc_fwd(const AttnShape& sh) { return g_path.load() == 0 && tc_fwd_supported(sh); }
 bool use_tc_bwd(const AttnShape& sh) { return g_path.load() == 0 && tc_bwd_supported(sh); }
 

@@ -50,6 +50,13 @@ bool tc_bwd_supported(const AttnShape& sh);
 
 int num_sms(int device);
 
+// The attention entry points' shape and argument rules (CPATTN_OK or the
+// status cpattn_fwd / cpattn_bwd would return), for callers that compose them.
+int check_attention_shape(int B, int H, int S, int D, int cp_size, int causal, float scale,
+                          int dtype);
+// Adds n kernels to the library's launch counter (cpattn_launch_count).
+void add_launches(int n);
+
 // Per-kernel timing for diagnostics: when enabled (cpattn_profile), every
 // launcher brackets each kernel with prof_begin / prof_end, which record a
 // pair of CUDA events on the launch stream.
@@ -63,7 +70,9 @@ enum KernelId : int {
   kKSimtDq = 6,
   kKTcDkdv = 7,
   kKTcDq = 8,
-  kKNumKernels = 9
+  kKLayerHeads = 9,   // head split / merge of the attention layer
+  kKLayerColsum = 10, // bias gradients of the attention layer
+  kKNumKernels = 11
 };
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);

@@ -94,3 +94,30 @@ def workload_inputs(w: Workload, with_dout=None):
     if with_dout is None:
         with_dout = w.backward
     return make_qkv(w.B, w.H, w.S, w.D, w.torch_dtype, w.seed, w.qkv_scale, with_dout)
+
+
+def make_layer_inputs(B, S, E, seed=0, dtype=torch.bfloat16):
+    """CPU tensors for the attention layer: x [B,S,E], w_qkv [3E,E], b_qkv [3E],
+    w_o [E,E], b_o [E], dy [B,S,E].  x and dy ~ N(0,1); weights and biases
+    ~ U(-1/sqrt(E), 1/sqrt(E)) (the range nn.Linear initialises them in), drawn
+    in that order from one seeded generator, then rounded to ``dtype``."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    bound = E ** -0.5
+
+    def uni(*shape):
+        return (torch.rand(shape, generator=g, dtype=torch.float32) * 2 - 1) * bound
+
+    x = torch.randn((B, S, E), generator=g, dtype=torch.float32)
+    w_qkv, b_qkv, w_o, b_o = uni(3 * E, E), uni(3 * E), uni(E, E), uni(E)
+    dy = torch.randn((B, S, E), generator=g, dtype=torch.float32)
+    return tuple(t.to(dtype) for t in (x, w_qkv, b_qkv, w_o, b_o, dy))
+
+
+def flops_layer(B, S, E, H, causal=True):
+    """Algorithmic FLOPs of one layer (forward, backward): projections
+    8*B*S*E^2 forward and twice that backward, plus the attention's counts."""
+    D = E // H
+    att = 4.0 * B * H * S * S * D * (0.5 if causal else 1.0)
+    proj = 8.0 * B * S * E * E
+    return proj + att, 2 * proj + 2.5 * att

@@ -98,6 +98,31 @@ def test_argument_errors_are_reported_before_launch(cp):
     assert cp.bwd_workspace_bytes(1, 1, 256, 96) == 0
 
 
+def test_layer_argument_errors_are_reported_before_launch(cp):
+    p = ctypes.c_void_p(256)
+    B, S, E, H = 1, 256, 256, 2
+    need = cp.layer_workspace_bytes(B, S, E, H)
+    assert need > 0 and cp.layer_workspace_bytes(B, S, 96, 1) == 0 and cp.layer_workspace_bytes(B, S, 256, 3) == 0
+
+    def fwd(ptr=p, S=S, E=E, H=H, cp_size=2, scale=0.1, ws=p, ws_bytes=need):
+        return cp.lib.cpattn_layer_fwd(*([ptr] + [p] * 10), B, S, E, H, cp_size, 1, scale, ws, ws_bytes, None)
+
+    def bwd(ptr=p, S=S, E=E, H=H, cp_size=2, ws_bytes=need):
+        return cp.lib.cpattn_layer_bwd(*([ptr] + [p] * 13), B, S, E, H, cp_size, 1, 0.1, p, ws_bytes, None)
+
+    assert fwd(E=96, H=1) == cp.ERR_SHAPE          # D = 96
+    assert fwd(E=256, H=3) == cp.ERR_SHAPE         # E not a multiple of H
+    assert fwd(ptr=None) == cp.ERR_ARG
+    assert fwd(ptr=ctypes.c_void_p(258)) == cp.ERR_ALIGN
+    assert fwd(scale=0.0) == cp.ERR_ARG
+    assert fwd(ws=None) == cp.ERR_WORKSPACE
+    assert fwd(ws_bytes=need - 1) == cp.ERR_WORKSPACE
+    assert fwd(S=100, ws_bytes=cp.layer_workspace_bytes(B, 100, E, H)) == cp.ERR_SHAPE  # chunk of 25 rows
+    assert bwd(ptr=None) == cp.ERR_ARG
+    assert bwd(ws_bytes=need - 1) == cp.ERR_WORKSPACE
+    assert bwd(cp_size=0) == cp.ERR_SHAPE
+
+
 def test_status_strings(cp):
     for s in range(8):
         assert cp.status_str(s)
