@@ -401,6 +401,27 @@ def run_gpu(args, w):
 LAYER_METRIC = "attention layer (projections + ring attention) TFLOP/s fwd+bwd on 1 B200"
 
 
+def layer_oracle_sample(w, seconds_hint=10.0):
+    """fp64 layer oracle (forward + backward) over the workload's layer shape
+    truncated to S' = 1024 rows.  Returns (TFLOP/s, description, threads)."""
+    from long_sequence_context_b200.inputs import flops_layer, make_layer_inputs
+    from oracle import layer as olayer
+    from oracle import oracle as orc
+    S_s, E = min(w.S, 1024), w.H * w.D
+    t = [a.double().numpy() for a in make_layer_inputs(1, S_s, E, seed=w.seed)]
+    flops = sum(flops_layer(1, S_s, E, w.H, w.causal))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        olayer.layer_bwd(*t, w.H, w.causal, w.scale)
+        reps += 1
+        total = time.perf_counter() - t0
+        if total >= seconds_hint or reps >= 20:
+            break
+    desc = (f"fp64 layer oracle fwd+bwd, B=1 S={S_s} E={E} H={w.H} (prefix length of the "
+            f"workload's shape), {reps} rep(s) in {total:.1f}s")
+    return flops * reps / total / 1e12, desc, orc.threads()
+
+
 def run_layer(args, w):
     """The attention layer around the ring attention, forward + backward per
     step: E = H * D of the workload, B, S, cp_size, causal as in it.  Separate
@@ -477,6 +498,10 @@ def run_layer(args, w):
             "gpu_launches": launches,
             "clocks": clk,
         }
+        if world == 1 and not args.no_cpu_baseline:
+            tfl, desc, threads = layer_oracle_sample(w)
+            line["cpu_baseline"] = {"value": tfl, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": desc}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

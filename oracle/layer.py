@@ -64,12 +64,13 @@ def layer_bwd(x, w_qkv, b_qkv, w_o, b_o, dy, H, causal, scale):
     """Returns dict with dx, dw_qkv, db_qkv, dw_o, db_o (and the forward's y)."""
     x, w_qkv, w_o, dy = map(_f64, (x, w_qkv, w_o, dy))
     y, c = layer_fwd(x, w_qkv, b_qkv, w_o, b_o, H, causal, scale)
-    dw_o = np.einsum("bsn,bsk->nk", dy, c["om"])
+    rows = lambda t: t.reshape(-1, t.shape[-1])
+    dw_o = rows(dy).T @ rows(c["om"])
     db_o = dy.sum(axis=(0, 1))
     dom = dy @ w_o
     dq, dk, dv = oracle.attn_bwd(c["q"], c["k"], c["v"], split_heads(dom, H), causal, scale)
     dqkv = np.concatenate([merge_heads(dq), merge_heads(dk), merge_heads(dv)], axis=-1)
-    dw_qkv = np.einsum("bsn,bsk->nk", dqkv, x)
+    dw_qkv = rows(dqkv).T @ rows(x)
     db_qkv = dqkv.sum(axis=(0, 1))
     dx = dqkv @ w_qkv
     return {"y": y, "dx": dx, "dw_qkv": dw_qkv, "db_qkv": db_qkv, "dw_o": dw_o, "db_o": db_o}
