@@ -38,8 +38,10 @@ TRAFFIC_FILES = {
     ("tc_dkdv", "causal_b1h32s32768d128_cp8_bf16"):
         os.path.join(ROOT, "profiles", "traffic_tc_dkdv_causal_b1h32s32768d128_cp8.txt"),
 }
+# the files whose contents determine the kernel's device code and its TMA boxes
+# (kernels.h only declares host launchers and profiling ids)
 KERNEL_SOURCES = {
-    "tc_dkdv": ["tc_bwd.cu", "bwd_common.cuh", "kernels.h", "sm100.cuh", "tmap.h", "ring.cuh"],
+    "tc_dkdv": ["tc_bwd.cu", "bwd_common.cuh", "sm100.cuh", "tmap.h", "ring.cuh"],
 }
 
 
