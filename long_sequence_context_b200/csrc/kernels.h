@@ -3,6 +3,8 @@
 // number of kernels it enqueued (>= 0) or -1 when a launch failed.
 #pragma once
 
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -56,6 +58,21 @@ int check_attention_shape(int B, int H, int S, int D, int cp_size, int causal, f
                           int dtype);
 // Adds n kernels to the library's launch counter (cpattn_launch_count).
 void add_launches(int n);
+
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per device (the attribute belongs to the device's copy of the
+// kernel); `done` holds one bit per device already set.
+template <typename Kernel>
+bool smem_attr_once(Kernel* func, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const unsigned long long bit = 1ull << dev;
+  if (done.load() & bit) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done.fetch_or(bit);
+  return true;
+}
 
 // Per-kernel timing for diagnostics: when enabled (cpattn_profile), every
 // launcher brackets each kernel with prof_begin / prof_end, which record a

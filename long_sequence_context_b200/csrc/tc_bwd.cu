@@ -475,13 +475,8 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.dk = static_cast<__nv_bfloat16*>(dk);
   P.dv = static_cast<__nv_bfloat16*>(dv);
   P.err = err;
-  static bool attr[2] = {false, false};
-  if (!attr[D == 128]) {
-    if (cudaFuncSetAttribute(tc_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DkdvCfg<D>::kSmemBytes) != cudaSuccess)
-      return -1;
-    attr[D == 128] = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(tc_dkdv_kernel<D>, DkdvCfg<D>::kSmemBytes, attr_done)) return -1;
   int dev = 0;
   cudaGetDevice(&dev);
   int grid = num_sms(dev);

@@ -389,13 +389,8 @@ template <int D>
 int launch_tc_dq(const BwdParams& P, const CUtensorMap& mq, const CUtensorMap& mk,
                  const CUtensorMap& mv, const CUtensorMap& mdo, int grid, cudaStream_t stream) {
   using C = DqCfg<D>;
-  static bool attr[2] = {false, false};
-  if (!attr[D == 128]) {
-    if (cudaFuncSetAttribute(tc_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return -1;
-    attr[D == 128] = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(tc_dq_kernel<D>, C::kSmemBytes, attr_done)) return -1;
   prof_begin(kKTcDq, stream);
   tc_dq_kernel<D><<<grid, 320, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
   prof_end(kKTcDq, stream);

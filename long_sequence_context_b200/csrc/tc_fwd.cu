@@ -543,13 +543,8 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.lse = lse;
   P.err = err;
   P.stall = stall;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[D == 128]) {
-    if (cudaFuncSetAttribute(tc_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return -1;
-    attr_set[D == 128] = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  if (!smem_attr_once(tc_fwd_kernel<D>, C::kSmemBytes, attr_done)) return -1;
   int dev = 0;
   cudaGetDevice(&dev);
   int grid = num_sms(dev);
