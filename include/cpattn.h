@@ -183,6 +183,16 @@ int cpattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* 
                        void* stream);
 
 /*
+ * cpattn_accumulate -- acc[i] += x[i] for i < n, acc fp32, x of `dtype`: the
+ * running gradient sums of the multi-rank ring backward, where every (q chunk,
+ * kv chunk) block adds its dQ, dK, dV terms ("Megatron-LM source analysis:
+ * Context Parallel", section 2: the backward mirrors the forward's exchange).
+ * n must be a multiple of 4 (CPATTN_ERR_SHAPE), both pointers 16-byte aligned
+ * (CPATTN_ERR_ALIGN); n = 0 does nothing.
+ */
+int cpattn_accumulate(float* acc, const void* x, long n, int dtype, void* stream);
+
+/*
  * The attention layer around the ring attention ("Configuring
  * RingAttention+FlashAttention for CP", section 3 code): Q, K, V projections
  * of width E (nn.Linear with bias), the [B,S,E] -> [B,H,S,D] head split, the
@@ -258,7 +268,8 @@ long long cpattn_launch_count(void);
  *   0 tcgen05 forward, 1 CUDA-core forward, 2 merge, 3 finalize, 4 backward
  *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 dK/dV,
  *   8 tcgen05 dQ, 9 layer head split / merge, 10 layer bias gradients (the
- *   layer's cuBLASLt GEMMs are not this library's kernels and are not timed).
+ *   layer's cuBLASLt GEMMs are not this library's kernels and are not timed),
+ *   11 gradient accumulation (cpattn_accumulate).
  */
 int cpattn_profile(int on);
 int cpattn_profile_read(int kernel_kind, double* total_ms, long long* launches);

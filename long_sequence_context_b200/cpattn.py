@@ -24,7 +24,8 @@ EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpat
            "cpattn_bwd_workspace_bytes", "cpattn_bwd", "cpattn_sync_status",
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
            "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc",
-           "cpattn_layer_workspace_bytes", "cpattn_layer_fwd", "cpattn_layer_bwd"]
+           "cpattn_layer_workspace_bytes", "cpattn_layer_fwd", "cpattn_layer_bwd",
+           "cpattn_accumulate"]
 
 # size of the library's fixed scratch array behind bwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -60,6 +61,7 @@ def _load():
         "cpattn_profile": ([i], i),
         "cpattn_profile_read": ([i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)], i),
         "cpattn_layer_workspace_bytes": ([i, i, i, i], sz),
+        "cpattn_accumulate": ([vp, vp, l, i, vp], i),
         "cpattn_layer_fwd": ([vp] * 11 + [i] * 6 + [f, vp, sz, vp], i),
         "cpattn_layer_bwd": ([vp] * 14 + [i] * 6 + [f, vp, sz, vp], i),
     }
@@ -209,6 +211,17 @@ def bwd_noalloc(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=
     return dq, dk, dv
 
 
+def accumulate_(acc, x, stream=None):
+    """acc += x (acc fp32, x bf16 or fp32, same number of elements)."""
+    if acc.dtype != torch.float32:
+        raise TypeError("acc must be fp32")
+    if acc.numel() != x.numel():
+        raise ValueError("acc and x must have the same number of elements")
+    _check(lib.cpattn_accumulate(_dev(acc, "acc"), _dev(x, "x"), acc.numel(), _dtype_code(x),
+                                 _stream(stream)), "cpattn_accumulate")
+    return acc
+
+
 def layer_workspace_bytes(B, S, E, H) -> int:
     return int(lib.cpattn_layer_workspace_bytes(B, S, E, H))
 
@@ -298,7 +311,7 @@ def debug_stall(n: int) -> int:
 
 KERNEL_KINDS = {0: "tc_fwd", 1: "simt_fwd", 2: "merge", 3: "finalize", 4: "bwd_delta",
                 5: "simt_dkdv", 6: "simt_dq", 7: "tc_dkdv", 8: "tc_dq", 9: "layer_heads",
-                10: "layer_colsum"}
+                10: "layer_colsum", 11: "accumulate"}
 
 
 def profile(on: bool) -> int:

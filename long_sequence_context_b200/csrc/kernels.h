@@ -89,7 +89,8 @@ enum KernelId : int {
   kKTcDq = 8,
   kKLayerHeads = 9,   // head split / merge of the attention layer
   kKLayerColsum = 10, // bias gradients of the attention layer
-  kKNumKernels = 11
+  kKAccumulate = 11,  // fp32 gradient sums of the multi-rank ring backward
+  kKNumKernels = 12
 };
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);

@@ -123,6 +123,16 @@ def test_layer_argument_errors_are_reported_before_launch(cp):
     assert bwd(cp_size=0) == cp.ERR_SHAPE
 
 
+def test_accumulate_argument_errors(cp):
+    p = ctypes.c_void_p(256)
+    assert cp.lib.cpattn_accumulate(p, p, 6, 0, None) == cp.ERR_SHAPE
+    assert cp.lib.cpattn_accumulate(p, p, -4, 0, None) == cp.ERR_SHAPE
+    assert cp.lib.cpattn_accumulate(p, p, 8, 7, None) == cp.ERR_DTYPE
+    assert cp.lib.cpattn_accumulate(None, p, 8, 0, None) == cp.ERR_ARG
+    assert cp.lib.cpattn_accumulate(p, ctypes.c_void_p(258), 8, 0, None) == cp.ERR_ALIGN
+    assert cp.lib.cpattn_accumulate(p, p, 0, 0, None) == cp.OK
+
+
 def test_status_strings(cp):
     for s in range(8):
         assert cp.status_str(s)
