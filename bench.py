@@ -567,6 +567,67 @@ def run_layer(args, w):
         dist.destroy_process_group()
 
 
+RING_METRIC = "ring attention across ranks (one sequence, chunks per GPU) TFLOP/s fwd+bwd"
+
+
+def run_ring(args, w):
+    """The multi-rank ring (long_sequence_context_b200/ring.py): one sequence of
+    the workload split over the N GPUs (2N zigzag chunks when causal), K/V
+    exchanged between neighbours every step; strong scaling (the total work is
+    the workload's).  Prints its own JSON line."""
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    from long_sequence_context_b200 import cpattn as cp
+    from long_sequence_context_b200 import ring
+    from long_sequence_context_b200.inputs import workload_inputs
+    dev = torch.device("cuda", local)
+    q, k, v, do = workload_inputs(w, with_dout=True)
+    loc = lambda x: [c.to(dev) for c in ring.local_chunks(x, rank, world, w.causal)]
+    ql, kl, vl, dol = loc(q), loc(k), loc(v), loc(do)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        o, lse = ring.ring_fwd(ql, kl, vl, w.causal, w.scale)
+        ring.ring_bwd(ql, kl, vl, o, lse, dol, w.causal, w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    if cp.sync_status() != cp.OK:
+        raise RuntimeError("ring warm-up failed")
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    n0 = cp.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = cp.launch_count() - n0
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world)
+    clk = clocks.stop()
+    if cp.sync_status() != cp.OK:
+        raise RuntimeError("ring timed region failed")
+    flops = w.flops_fwd() + w.flops_bwd()
+    if rank == 0:
+        line = {"metric": RING_METRIC, "value": flops / (ms_total / args.steps * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_total / args.steps, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"ring_{w.name}", "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                           "ring_ranks": world, "causal": w.causal,
+                           "chunk_rows": w.S // (2 * world if w.causal else world)},
+                "gpu_launches": launches, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -577,6 +638,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fwd-only", action="store_true", help="time the forward alone (profiling)")
+    ap.add_argument("--ring", action="store_true",
+                    help="time the multi-rank ring: one sequence split over the --gpus ranks")
     ap.add_argument("--layer", action="store_true",
                     help="time the attention layer (projections + ring attention) instead")
     ap.add_argument("--shape", default=None,
@@ -595,6 +658,8 @@ def main():
         run_reference(args, w)
     elif args.layer:
         run_layer(args, w)
+    elif args.ring:
+        run_ring(args, w)
     else:
         run_gpu(args, w)
 

@@ -220,19 +220,26 @@ def run_loopback(gens):
             raise RuntimeError("ranks out of step")
 
 
-def ring_fwd(q, k, v, causal=True, scale=None, group=None):
-    """Ring forward of this rank over torch.distributed: q, k, v are its chunk
-    tensors (local_chunks order).  Returns lists (o, lse) per own chunk."""
+def _drive(make_gen, group):
+    """Run a schedule over torch.distributed, or as a single rank when no
+    process group is initialised (no exchanges then)."""
     import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        return run_dist(make_gen(dist.get_rank(group), dist.get_world_size(group)), group)
+    return run_loopback([make_gen(0, 1)])[0]
+
+
+def ring_fwd(q, k, v, causal=True, scale=None, group=None):
+    """Ring forward of this rank: q, k, v are its chunk tensors (local_chunks
+    order).  Returns lists (o, lse) per own chunk."""
     scale = float(scale if scale is not None else q[0].shape[-1] ** -0.5)
-    out = run_dist(fwd_schedule(dist.get_rank(group), dist.get_world_size(group), q, k, v, causal,
-                                CudaBlocks(scale)), group)
+    be = CudaBlocks(scale)
+    out = _drive(lambda r, n: fwd_schedule(r, n, q, k, v, causal, be), group)
     return [o for o, _ in out], [l for _, l in out]
 
 
 def ring_bwd(q, k, v, o, lse, do, causal=True, scale=None, group=None):
     """Ring backward of this rank: returns lists (dq, dk, dv) per own chunk."""
-    import torch.distributed as dist
     scale = float(scale if scale is not None else q[0].shape[-1] ** -0.5)
-    return run_dist(bwd_schedule(dist.get_rank(group), dist.get_world_size(group), q, k, v, o, lse,
-                                 do, causal, CudaBlocks(scale)), group)
+    be = CudaBlocks(scale)
+    return _drive(lambda r, n: bwd_schedule(r, n, q, k, v, o, lse, do, causal, be), group)
