@@ -1,0 +1,27 @@
+"""CPU checks of bench.py's bookkeeping: the recorded DRAM traffic is reported
+only while the kernel's sources match the digest stored with the capture."""
+import bench
+
+
+def _write(tmp_path, digest, value=123456):
+    p = tmp_path / "traffic.txt"
+    p.write_text("# a comment line: with a colon\n"
+                 f"kernel: tc_dkdv\nworkload: w\ndram_bytes_per_launch: {value}\nsource_sha256: {digest}\n")
+    return str(p)
+
+
+def test_recorded_traffic_needs_matching_sources(tmp_path, monkeypatch):
+    good = _write(tmp_path, bench.kernel_source_digest("tc_dkdv"))
+    monkeypatch.setitem(bench.TRAFFIC_FILES, ("tc_dkdv", "w"), good)
+    assert bench.recorded_traffic("tc_dkdv", "w") == 123456
+    stale = _write(tmp_path, "0" * 64)
+    monkeypatch.setitem(bench.TRAFFIC_FILES, ("tc_dkdv", "w"), stale)
+    assert bench.recorded_traffic("tc_dkdv", "w") is None
+    assert bench.recorded_traffic("tc_dq", "w") is None            # no capture recorded
+    assert bench.recorded_traffic("tc_dkdv", "other") is None
+
+
+def test_digest_covers_the_listed_sources():
+    d = bench.kernel_source_digest("tc_dkdv")
+    assert len(d) == 64 and d == bench.kernel_source_digest("tc_dkdv")
+    assert "tc_bwd.cu" in bench.KERNEL_SOURCES["tc_dkdv"]
