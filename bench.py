@@ -255,6 +255,110 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------- standalone LSE merge --
+MERGE_ROWS, MERGE_D = 1 << 20, 128
+
+
+def merge_bytes_per_row(D):
+    """Algorithmic bytes of one merged row: read O_acc, O_part (D fp32 each) and
+    the two LSEs, write O_acc and LSE_acc."""
+    return 3 * D * 4 + 3 * 4
+
+
+def time_merge(cp, dev, peaks, launches=20, warmup=3, rows=MERGE_ROWS, D=MERGE_D):
+    """cpattn_merge over `rows` rows of D fp32 (in place, the same buffers every
+    launch; 1.6 GB of operands, far larger than L2): mean device time per launch
+    from CUDA events on the launch stream, GB/s of algorithmic bytes."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(77)
+    o_acc = torch.randn((rows, D), generator=g, device=dev)
+    o_part = torch.randn((rows, D), generator=g, device=dev)
+    lse_acc = torch.randn((rows,), generator=g, device=dev)
+    lse_part = torch.randn((rows,), generator=g, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        cp.merge_(o_acc, lse_acc, o_part, lse_part)
+    torch.cuda.synchronize(dev)
+    n0 = cp.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(launches):
+        cp.merge_(o_acc, lse_acc, o_part, lse_part)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    n = cp.launch_count() - n0
+    ms = e0.elapsed_time(e1) / launches
+    per_launch = merge_bytes_per_row(D) * rows
+    gbs = per_launch / (ms * 1e-3) / 1e9
+    st = cp.sync_status()
+    if st != cp.OK:
+        raise RuntimeError(f"merge failed: {cp.status_str(st)}")
+    del o_acc, o_part, lse_acc, lse_part
+    return {"kernel": "merge_kernel", "rows": rows, "D": D, "launches": n,
+            "ms_per_launch": ms, "bytes_per_launch": per_launch,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"],
+                         "peak_kind": f"hbm_gbs ({peaks['source']})"}}
+
+
+def time_workload(cp, w, dev, peaks, steps=5, warmup=3):
+    """Device time of one workload's hot path (forward, plus backward when the
+    workload has one), per kernel from the library's event hooks."""
+    import torch
+    from long_sequence_context_b200.inputs import workload_inputs
+    q, k, v, do = (t.to(dev) for t in workload_inputs(w, with_dout=True))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    grads = [torch.empty_like(q) for _ in range(3)]
+    ws = torch.empty(cp.bwd_workspace_bytes(w.B, w.H, w.S, w.D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cp.fwd(q, k, v, w.cp_size, w.causal, w.scale, out=o, lse=lse)
+        if w.backward:
+            cp.bwd(q, k, v, o, lse, do, w.cp_size, w.causal, w.scale, workspace=ws,
+                   dq=grads[0], dk=grads[1], dv=grads[2])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    cp.profile(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    cp.profile(False)
+    st = cp.sync_status()
+    if st != cp.OK:
+        raise RuntimeError(f"{w.name} failed: {cp.status_str(st)}")
+    ms = e0.elapsed_time(e1) / steps
+    kern = {}
+    for kind, name in cp.KERNEL_KINDS.items():
+        t, n = cp.profile_read(kind)
+        if n:
+            kern[name] = t / steps
+    fwd_ms = kern.get("tc_fwd", kern.get("simt_fwd"))
+    f_fwd = w.flops_fwd()
+    f_bwd = w.flops_bwd() if w.backward else 0.0
+    bwd_ms = (ms - fwd_ms) if (w.backward and fwd_ms) else None
+    del q, k, v, do, o, lse, grads, ws
+    torch.cuda.empty_cache()
+    out = {"passes": "fwd+bwd" if w.backward else "fwd", "dtype": w.dtype,
+           "ms_per_step": ms, "tflops": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12,
+           "fwd_ms": fwd_ms, "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12 if fwd_ms else None,
+           "kernel_ms_per_step": kern}
+    if w.backward and bwd_ms:
+        out["bwd_ms"] = bwd_ms
+        out["bwd_tflops"] = f_bwd / (bwd_ms * 1e-3) / 1e12
+    if w.dtype == "bf16":
+        out["frac_of_peak"] = out["tflops"] / peaks["bf16_tflops"]
+        if fwd_ms:
+            out["fwd_frac_of_peak"] = out["fwd_tflops"] / peaks["bf16_tflops"]
+    return out
+
+
 # --------------------------------------------------------------- GPU arm --
 def run_gpu(args, w):
     import torch
@@ -424,6 +528,17 @@ def run_gpu(args, w):
                "serial": {"value": job_tflops(f_fwd + f_bwd, n_e2e, ser_ms, world),
                           "ms_per_step": ser_ms / n_e2e}}
 
+    # ---- the other workloads and the standalone merge (device-timed, after the
+    # headline region; each its own allocation) ----
+    per_config, merge = None, None
+    if not args.no_extra and world == 1:
+        per_config = {}
+        from long_sequence_context_b200.inputs import WORKLOADS
+        for name, wk in WORKLOADS.items():
+            if name != w.name:
+                per_config[name] = time_workload(cp, wk, dev, peaks)
+        merge = time_merge(cp, dev, peaks)
+
     # ---- CPU baseline: the oracle on this host, rank 0, N == 1 only ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -446,6 +561,8 @@ def run_gpu(args, w):
             "peaks": peaks,
             "per_kernel_ms": per_kernel,
             "roofline": roof,
+            "per_config": per_config,
+            "merge": merge,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
@@ -628,6 +745,36 @@ def run_ring(args, w):
         dist.destroy_process_group()
 
 
+MERGE_METRIC = "standalone LSE merge (cpattn_merge) GB/s on 1 B200; fraction of measured HBM copy bandwidth"
+
+
+def run_merge(args):
+    """The standalone log-sum-exp merge of two fp32 partials over 1,048,576 rows
+    of D = 128 (one S = 32K, H = 32 set of rows).  Prints its own JSON line."""
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    from long_sequence_context_b200 import cpattn as cp
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    m = time_merge(cp, dev, peaks, launches=args.steps, warmup=args.warmup)
+    clk = clocks.stop()
+    if rank == 0:
+        line = {"metric": MERGE_METRIC, "value": m["roofline"]["achieved"], "unit": "GB/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": m["ms_per_launch"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": f"merge_rows{m['rows']}_d{m['D']}", "rows": m["rows"], "D": m["D"],
+                           "l2": "operands 1.6 GB, larger than L2; no flush"},
+                "roofline": m["roofline"], "gpu_launches": m["launches"], "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -642,6 +789,10 @@ def main():
                     help="time the multi-rank ring: one sequence split over the --gpus ranks")
     ap.add_argument("--layer", action="store_true",
                     help="time the attention layer (projections + ring attention) instead")
+    ap.add_argument("--merge", action="store_true",
+                    help="time the standalone LSE merge (cpattn_merge) alone")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads and the merge in the headline line")
     ap.add_argument("--shape", default=None,
                     help="B,H,S,D,cp_size,causal: a smaller case of the workload (profiling)")
     args = ap.parse_args()
@@ -656,6 +807,8 @@ def main():
                                 cp_size=N, causal=bool(c))
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.merge:
+        run_merge(args)
     elif args.layer:
         run_layer(args, w)
     elif args.ring:

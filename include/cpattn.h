@@ -40,6 +40,11 @@
  *     rest on the CUDA-core kernels.
  *   - Pointers must be 16-byte aligned (CPATTN_ERR_ALIGN); scale must be
  *     finite and > 0 (CPATTN_ERR_ARG).
+ *   - Sizes are not visible through plain pointers: every buffer must hold the
+ *     elements its stated layout implies (the Python binding checks shapes and
+ *     dtypes before calling).
+ *   - Each entry point opens an NVTX range named after itself for the host
+ *     side of the call (no-op without an attached profiler).
  */
 #ifndef CPATTN_H
 #define CPATTN_H
@@ -151,6 +156,29 @@ int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const
                int cp_size, int causal, float scale, void* workspace, size_t ws_bytes,
                int dtype, void* stream);
 
+/*
+ * cpattn_bwd_accumulate -- the same backward as cpattn_bwd, but the block's
+ * gradients are ADDED, in fp32 and without rounding to the input dtype, into
+ * caller-owned fp32 accumulators:
+ *     dq_acc += dQ,  dk_acc += dK,  dv_acc += dV      ([B][H][S][D] fp32 each)
+ * For the multi-rank ring and all-gather drivers, which call the backward once
+ * per (q chunk, kv chunk) block and sum the blocks' terms for every chunk
+ * ("Megatron-LM source analysis: Context Parallel", section 2: the backward
+ * mirrors the forward's exchange, every block adding to the gradients of its q
+ * and kv chunks).  With bf16 inputs the sums then carry one rounding at the
+ * end (the caller's cast) instead of one per block term.
+ *   Arguments, workspace, preconditions and errors: as cpattn_bwd.  The
+ *   accumulators must not alias each other or any input.  Every element of
+ *   every accumulator is read and written exactly once per call (no atomics), so
+ *   calls on one stream compose; calls that overlap on the GPU and share an
+ *   accumulator race.
+ */
+int cpattn_bwd_accumulate(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, float* dq_acc, float* dk_acc,
+                          float* dv_acc, int B, int H, int S, int D, int cp_size, int causal,
+                          float scale, void* workspace, size_t ws_bytes, int dtype,
+                          void* stream);
+
 /* Size of the fixed device scratch array used by cpattn_bwd_noalloc (64 MiB). */
 #define CPATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
 
@@ -170,12 +198,18 @@ int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const
  *   CPATTN_NOALLOC_SCRATCH_BYTES are rejected with CPATTN_ERR_WORKSPACE before
  *   anything is enqueued (CPATTN_ERR_SHAPE for invalid sizes).
  *   Set-up: the first call on a device looks up the array's device address
- *   (with that device current); make that first call before any stream
- *   capture begins.
+ *   (with that device current) and keeps it for the life of the process;
+ *   make that first call before any stream capture begins.  The address
+ *   belongs to the device's current context: do not use the library across a
+ *   cudaDeviceReset (or any other teardown of the primary context) in the same
+ *   process.
  *   Sharing: all calls on a device use the same array, which keeps the last
- *   call's contents (the backward clears what it accumulates into).  Calls
- *   that can overlap on the GPU -- on different streams, or from different
- *   host threads -- race on the array; serialise them.
+ *   call's contents.  It holds two fp32 values per row, delta_i = dO_i . O_i
+ *   and LSE_i * log2(e); the backward's preprocess kernel rewrites both for
+ *   every row of the call before anything reads them, so leftovers of earlier
+ *   calls are never used (dQ, dK and dV go straight to the caller's outputs).
+ *   Calls that can overlap on the GPU -- on different streams, or from
+ *   different host threads -- race on the array; serialise them.
  */
 int cpattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
@@ -236,7 +270,9 @@ int cpattn_layer_bwd(const void* x, const void* w_qkv, const void* w_o, const vo
 /*
  * cpattn_sync_status -- synchronises `stream`, then returns and clears the
  * device-side error word of the current device (CPATTN_OK, CPATTN_ERR_TIMEOUT)
- * or CPATTN_ERR_CUDA if the synchronisation itself failed.
+ * or CPATTN_ERR_CUDA if the synchronisation itself failed.  The word's device
+ * address is looked up once per device and kept: as for cpattn_bwd_noalloc,
+ * do not use the library across a cudaDeviceReset in the same process.
  */
 int cpattn_sync_status(void* stream);
 

@@ -65,10 +65,8 @@ def allgather_bwd_blocks(rank, world, q, k_all, v_all, o, lse, do, causal, be):
             kind = ring.block_kind(a, b, causal)
             if kind == ring.SKIP:
                 continue
-            gq, gk, gv = be.bwd(q[ai], k_all[b], v_all[b], o[ai], lse[ai], do[ai], kind == ring.DIAG)
-            be.accumulate(dq[ai], gq)
-            be.accumulate(dk[b], gk)
-            be.accumulate(dv[b], gv)
+            be.bwd_into(q[ai], k_all[b], v_all[b], o[ai], lse[ai], do[ai], kind == ring.DIAG,
+                        dq[ai], dk[b], dv[b])
     return dq, dk, dv
 
 

@@ -25,7 +25,7 @@ EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpat
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
            "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc",
            "cpattn_layer_workspace_bytes", "cpattn_layer_fwd", "cpattn_layer_bwd",
-           "cpattn_accumulate"]
+           "cpattn_accumulate", "cpattn_bwd_accumulate"]
 
 # size of the library's fixed scratch array behind bwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -51,6 +51,7 @@ def _load():
         "cpattn_finalize": ([vp, vp, l, i, i, vp], i),
         "cpattn_bwd_workspace_bytes": ([i, i, i, i], sz),
         "cpattn_bwd": ([vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, sz, i, vp], i),
+        "cpattn_bwd_accumulate": ([vp] * 9 + [i, i, i, i, i, i, f, vp, sz, i, vp], i),
         "cpattn_sync_status": ([vp], i),
         "cpattn_status_str": ([i], ctypes.c_char_p),
         "cpattn_launch_count": ([], ctypes.c_longlong),
@@ -99,11 +100,40 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _dev(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _expect(t, name: str, shape, dtype, like=None):
+    """Shape / dtype / device check of one tensor argument.  The C ABI sees
+    plain pointers, so a wrong-sized buffer would be read or written out of
+    bounds on the device: every tensor is checked here before any call."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if like is not None and t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, expected {like.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _qkv(q, k, v):
+    """Checks q, k, v ([B, H, S, D], one dtype, one device); returns the shape."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a [B, H, S, D] tensor")
+    _dtype_code(q)
+    for t, n in ((k, "k"), (v, "v")):
+        _expect(t, n, q.shape, q.dtype, q)
+    _expect(q, "q", q.shape, q.dtype)
+    return tuple(q.shape)
 
 
 def plan(S: int, cp_size: int, causal: bool):
@@ -120,13 +150,14 @@ def plan(S: int, cp_size: int, causal: bool):
 
 def fwd(q, k, v, cp_size: int, causal: bool = True, scale=None, out=None, lse=None, stream=None):
     """Ring forward: returns (o, lse) with o like q and lse fp32 [B, H, S]."""
-    B, H, S, D = q.shape
+    B, H, S, D = _qkv(q, k, v)
     scale = float(scale if scale is not None else D ** -0.5)
+    if out is not None:
+        _expect(out, "out", q.shape, q.dtype, q)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, S), torch.float32, q)
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if lse is None else lse
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        if t.shape != q.shape or t.dtype != q.dtype:
-            raise ValueError(f"{n} must match q in shape and dtype")
     st = lib.cpattn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse_t, "lse"),
                         B, H, S, D, cp_size, int(causal), scale, _dtype_code(q), _stream(stream))
     _check(st, "cpattn_fwd")
@@ -135,7 +166,7 @@ def fwd(q, k, v, cp_size: int, causal: bool = True, scale=None, out=None, lse=No
 
 def fwd_step(q, k, v, cp_size: int, step: int, causal: bool = True, scale=None, stream=None):
     """One ring step for every virtual rank: fp32 partial (o_part, lse_part)."""
-    B, H, S, D = q.shape
+    B, H, S, D = _qkv(q, k, v)
     scale = float(scale if scale is not None else D ** -0.5)
     o = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
@@ -147,12 +178,17 @@ def fwd_step(q, k, v, cp_size: int, step: int, causal: bool = True, scale=None, 
 
 
 def merge_(o_acc, lse_acc, o_part, lse_part, stream=None):
-    """In-place log-sum-exp merge of (o_part, lse_part) into (o_acc, lse_acc)."""
+    """In-place log-sum-exp merge of (o_part, lse_part) into (o_acc, lse_acc):
+    o tensors [..., D] fp32, lse tensors the same leading shape, fp32."""
+    if not isinstance(o_acc, torch.Tensor) or o_acc.dim() < 1:
+        raise ValueError("o_acc must be a [..., D] tensor")
     D = o_acc.shape[-1]
+    lead = tuple(o_acc.shape[:-1])
+    _expect(o_acc, "o_acc", o_acc.shape, torch.float32)
+    _expect(lse_acc, "lse_acc", lead, torch.float32, o_acc)
+    _expect(o_part, "o_part", o_acc.shape, torch.float32, o_acc)
+    _expect(lse_part, "lse_part", lead, torch.float32, o_acc)
     rows = lse_acc.numel()
-    for t in (o_acc, lse_acc, o_part, lse_part):
-        if t.dtype != torch.float32:
-            raise TypeError("merge operands are fp32")
     st = lib.cpattn_merge(_dev(o_acc, "o_acc"), _dev(lse_acc, "lse_acc"), _dev(o_part, "o_part"),
                           _dev(lse_part, "lse_part"), rows, D, _stream(stream))
     _check(st, "cpattn_merge")
@@ -160,6 +196,10 @@ def merge_(o_acc, lse_acc, o_part, lse_part, stream=None):
 
 
 def finalize(o_acc, dtype=torch.bfloat16, stream=None):
+    """fp32 [..., D] -> a new tensor of `dtype` (round to nearest even)."""
+    if not isinstance(o_acc, torch.Tensor) or o_acc.dim() < 1:
+        raise ValueError("o_acc must be a [..., D] tensor")
+    _expect(o_acc, "o_acc", o_acc.shape, torch.float32)
     D = o_acc.shape[-1]
     o = torch.empty(o_acc.shape, dtype=dtype, device=o_acc.device)
     st = lib.cpattn_finalize(_dev(o_acc, "o_acc"), _dev(o, "o"), o_acc.numel() // D, D,
@@ -172,14 +212,34 @@ def bwd_workspace_bytes(B, H, S, D) -> int:
     return int(lib.cpattn_bwd_workspace_bytes(B, H, S, D))
 
 
+def _bwd_args(q, k, v, o, lse, dout):
+    B, H, S, D = _qkv(q, k, v)
+    _expect(o, "o", q.shape, q.dtype, q)
+    _expect(dout, "dout", q.shape, q.dtype, q)
+    _expect(lse, "lse", (B, H, S), torch.float32, q)
+    return B, H, S, D
+
+
+def _workspace(workspace, need, q):
+    if workspace is None:
+        return torch.empty(need, dtype=torch.uint8, device=q.device)
+    if not isinstance(workspace, torch.Tensor) or workspace.device != q.device:
+        raise ValueError(f"workspace must be a tensor on {q.device}")
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace holds {workspace.numel() * workspace.element_size()} bytes, "
+                         f"{need} needed")
+    return workspace
+
+
 def bwd(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=None, workspace=None,
         dq=None, dk=None, dv=None, stream=None):
     """Recompute backward: returns (dq, dk, dv) like q."""
-    B, H, S, D = q.shape
+    B, H, S, D = _bwd_args(q, k, v, o, lse, dout)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if t is not None:
+            _expect(t, n, q.shape, q.dtype, q)
     scale = float(scale if scale is not None else D ** -0.5)
-    need = bwd_workspace_bytes(B, H, S, D)
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    workspace = _workspace(workspace, bwd_workspace_bytes(B, H, S, D), q)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
@@ -192,13 +252,36 @@ def bwd(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=None, wo
     return dq, dk, dv
 
 
+def bwd_accumulate_(q, k, v, o, lse, dout, dq_acc, dk_acc, dv_acc, cp_size: int,
+                    causal: bool = True, scale=None, workspace=None, stream=None):
+    """Recompute backward whose gradients are added, in fp32, into the fp32
+    accumulators dq_acc, dk_acc, dv_acc (each shaped like q).  Returns them."""
+    B, H, S, D = _bwd_args(q, k, v, o, lse, dout)
+    for t, n in ((dq_acc, "dq_acc"), (dk_acc, "dk_acc"), (dv_acc, "dv_acc")):
+        _expect(t, n, q.shape, torch.float32, q)
+    if len({dq_acc.data_ptr(), dk_acc.data_ptr(), dv_acc.data_ptr()}) != 3:
+        raise ValueError("dq_acc, dk_acc, dv_acc must be distinct tensors")
+    scale = float(scale if scale is not None else D ** -0.5)
+    workspace = _workspace(workspace, bwd_workspace_bytes(B, H, S, D), q)
+    st = lib.cpattn_bwd_accumulate(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"),
+        _dev(dout, "dout"), _dev(dq_acc, "dq_acc"), _dev(dk_acc, "dk_acc"), _dev(dv_acc, "dv_acc"),
+        B, H, S, D, cp_size, int(causal), scale, ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream))
+    _check(st, "cpattn_bwd_accumulate")
+    return dq_acc, dk_acc, dv_acc
+
+
 def bwd_noalloc(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=None,
                 dq=None, dk=None, dv=None, stream=None):
     """Backward without a caller workspace: the library's fixed device scratch
     array stands in for it (see cpattn_bwd_noalloc in include/cpattn.h).  For
     callers that cannot allocate device memory, pass preallocated dq/dk/dv;
     calls that may overlap on the GPU must be serialised by the caller."""
-    B, H, S, D = q.shape
+    B, H, S, D = _bwd_args(q, k, v, o, lse, dout)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if t is not None:
+            _expect(t, n, q.shape, q.dtype, q)
     scale = float(scale if scale is not None else D ** -0.5)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
@@ -212,11 +295,12 @@ def bwd_noalloc(q, k, v, o, lse, dout, cp_size: int, causal: bool = True, scale=
 
 
 def accumulate_(acc, x, stream=None):
-    """acc += x (acc fp32, x bf16 or fp32, same number of elements)."""
-    if acc.dtype != torch.float32:
-        raise TypeError("acc must be fp32")
-    if acc.numel() != x.numel():
-        raise ValueError("acc and x must have the same number of elements")
+    """acc += x (acc fp32, x bf16 or fp32, same shape)."""
+    _expect(acc, "acc", acc.shape, torch.float32)
+    if not isinstance(x, torch.Tensor):
+        raise TypeError("x must be a torch.Tensor")
+    _dtype_code(x)
+    _expect(x, "x", acc.shape, x.dtype, acc)
     _check(lib.cpattn_accumulate(_dev(acc, "acc"), _dev(x, "x"), acc.numel(), _dtype_code(x),
                                  _stream(stream)), "cpattn_accumulate")
     return acc
@@ -266,6 +350,7 @@ def layer_bwd(x, w_qkv, w_o, saved, dy, num_heads: int, cp_size: int, causal: bo
     D = E // H
     scale = float(scale if scale is not None else D ** -0.5)
     q, k, v, o, lse = saved
+    _expect(lse, "lse", (B, H, S), torch.float32, x)
     if workspace is None:
         workspace = torch.empty(layer_workspace_bytes(B, S, E, H), dtype=torch.uint8, device=x.device)
     dx = torch.empty_like(x)

@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(256) accumulate_kernel(float* __restrict__ acc
 using namespace cpattn;
 
 extern "C" int cpattn_accumulate(float* acc, const void* x, long n, int dtype, void* stream) {
+  NvtxRange nv("cpattn_accumulate");
   if (dtype != CPATTN_BF16 && dtype != CPATTN_FP32) return CPATTN_ERR_DTYPE;
   if (n < 0 || n % 4 != 0) return CPATTN_ERR_SHAPE;
   if (n == 0) return CPATTN_OK;

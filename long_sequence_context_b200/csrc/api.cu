@@ -127,6 +127,7 @@ int cpattn_last_path(void) { return g_last_path.load(); }
 int cpattn_debug_stall(int n) { return g_stall.exchange(n < 0 ? 0 : n); }
 
 int cpattn_plan(int S, int cp_size, int causal, int32_t* out, int capacity, int* n_rows) {
+  NvtxRange nv("cpattn_plan");
   if (!n_rows) return CPATTN_ERR_ARG;
   *n_rows = 0;
   if (cp_size < 1 || S < 1) return CPATTN_ERR_SHAPE;
@@ -157,6 +158,7 @@ int cpattn_plan(int S, int cp_size, int causal, int32_t* out, int capacity, int*
 
 int cpattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int S, int D, int cp_size, int causal, float scale, int dtype, void* stream) {
+  NvtxRange nv("cpattn_fwd");
   AttnShape sh;
   int st = check_shape(B, H, S, D, cp_size, causal, scale, dtype, &sh);
   if (st) return st;
@@ -182,6 +184,7 @@ int cpattn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 int cpattn_fwd_step(const void* q, const void* k, const void* v, float* o_part,
                     float* lse_part, int B, int H, int S, int D, int cp_size, int causal,
                     float scale, int step, int dtype, void* stream) {
+  NvtxRange nv("cpattn_fwd_step");
   AttnShape sh;
   int st = check_shape(B, H, S, D, cp_size, causal, scale, dtype, &sh);
   if (st) return st;
@@ -203,6 +206,7 @@ int cpattn_fwd_step(const void* q, const void* k, const void* v, float* o_part,
 
 int cpattn_merge(float* o_acc, float* lse_acc, const float* o_part, const float* lse_part,
                  long rows, int D, void* stream) {
+  NvtxRange nv("cpattn_merge");
   if (rows < 0) return CPATTN_ERR_SHAPE;
   if (D != 64 && D != 128) return CPATTN_ERR_SHAPE;
   if (rows == 0) return CPATTN_OK;
@@ -213,6 +217,7 @@ int cpattn_merge(float* o_acc, float* lse_acc, const float* o_part, const float*
 }
 
 int cpattn_finalize(const float* o_acc, void* o, long rows, int D, int dtype, void* stream) {
+  NvtxRange nv("cpattn_finalize");
   if (dtype != CPATTN_BF16 && dtype != CPATTN_FP32) return CPATTN_ERR_DTYPE;
   if (rows < 0) return CPATTN_ERR_SHAPE;
   if (D != 64 && D != 128) return CPATTN_ERR_SHAPE;
@@ -231,10 +236,16 @@ size_t cpattn_bwd_workspace_bytes(int B, int H, int S, int D) {
   return 2 * one;
 }
 
-int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-               const void* dout, void* dq, void* dk, void* dv, int B, int H, int S, int D,
-               int cp_size, int causal, float scale, void* workspace, size_t ws_bytes,
-               int dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// cpattn_bwd and cpattn_bwd_accumulate: the same backward; acc_f32 != 0 adds
+// the gradients into fp32 accumulators instead of writing them.
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+             int cp_size, int causal, float scale, void* workspace, size_t ws_bytes, int dtype,
+             int acc_f32, void* stream) {
   AttnShape sh;
   int st = check_shape(B, H, S, D, cp_size, causal, scale, dtype, &sh);
   if (st) return st;
@@ -254,13 +265,38 @@ int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (use_tc_bwd(sh)) {
     g_last_path = 0;
-    return count(launch_tc_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, s));
+    return count(
+        launch_tc_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, acc_f32, err, s));
   }
   g_last_path = 1;
-  return count(launch_simt_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, s));
+  return count(launch_simt_bwd(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, acc_f32, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int cpattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, int B, int H, int S, int D,
+               int cp_size, int causal, float scale, void* workspace, size_t ws_bytes,
+               int dtype, void* stream) {
+  NvtxRange nv("cpattn_bwd");
+  return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, S, D, cp_size, causal, scale,
+                  workspace, ws_bytes, dtype, 0, stream);
+}
+
+int cpattn_bwd_accumulate(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, float* dq_acc, float* dk_acc,
+                          float* dv_acc, int B, int H, int S, int D, int cp_size, int causal,
+                          float scale, void* workspace, size_t ws_bytes, int dtype,
+                          void* stream) {
+  NvtxRange nv("cpattn_bwd_accumulate");
+  return bwd_impl(q, k, v, o, lse, dout, dq_acc, dk_acc, dv_acc, B, H, S, D, cp_size, causal,
+                  scale, workspace, ws_bytes, dtype, 1, stream);
 }
 
 int cpattn_sync_status(void* stream) {
+  NvtxRange nv("cpattn_sync_status");
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return CPATTN_ERR_CUDA;
   unsigned* err = err_word();

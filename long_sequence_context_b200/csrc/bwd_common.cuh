@@ -33,6 +33,12 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  // accumulate mode (acc_f32 != 0): the gradients are added in fp32 into
+  // these [BH][S][D] arrays instead of being written to dq / dk / dv
+  int acc_f32;
+  float* dq_acc;
+  float* dk_acc;
+  float* dv_acc;
   unsigned* err;
 };
 
@@ -145,6 +151,22 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
   for (int c = 0; c < 4; ++c)
     d4[c] = make_uint4(pack_scaled(v[8 * c], v[8 * c + 1], mul), pack_scaled(v[8 * c + 2], v[8 * c + 3], mul),
                        pack_scaled(v[8 * c + 4], v[8 * c + 5], mul), pack_scaled(v[8 * c + 6], v[8 * c + 7], mul));
+}
+
+// Add 32 fp32 TMEM values (scaled) into an fp32 row of global memory.  Every
+// output row belongs to one thread of one work item, so the read-modify-write
+// needs no atomics; launches on one stream are ordered.
+__device__ __forceinline__ void add_row32(float* dst, const uint32_t (&v)[32], float mul) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float4 a = d4[c];
+    a.x += __uint_as_float(v[4 * c]) * mul;
+    a.y += __uint_as_float(v[4 * c + 1]) * mul;
+    a.z += __uint_as_float(v[4 * c + 2]) * mul;
+    a.w += __uint_as_float(v[4 * c + 3]) * mul;
+    d4[c] = a;
+  }
 }
 
 }  // namespace bwd

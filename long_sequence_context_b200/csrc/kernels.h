@@ -6,6 +6,7 @@
 #include <atomic>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -32,9 +33,10 @@ int launch_finalize(const float* o_acc, void* o, long rows, int D, int bf16,
                     cudaStream_t stream);
 // backward: delta = rowsum(dO * O) into ws_delta, then dK/dV (key-owned) and
 // dQ (row-owned) kernels; no atomics.
+// acc_f32 != 0: dq / dk / dv are fp32 accumulators the gradients are added to
 int launch_simt_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                     const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                    void* dv, float* ws_delta, cudaStream_t stream);
+                    void* dv, float* ws_delta, int acc_f32, cudaStream_t stream);
 
 // ---- tcgen05 tensor-core kernels (bf16, D in {64,128}, chunk % 128 == 0) ----
 int launch_tc_fwd(const AttnShape& sh, const void* q, const void* k, const void* v, void* o,
@@ -43,10 +45,12 @@ int launch_tc_fwd(const AttnShape& sh, const void* q, const void* k, const void*
 int launch_tc_fwd_step(const AttnShape& sh, const void* q, const void* k, const void* v,
                        float* o_part, float* lse_part, int step, unsigned* err,
                        cudaStream_t stream);
-// workspace: per-row delta and LSE * log2(e), fp32 [B*H*S] each
+// workspace: per-row delta and LSE * log2(e), fp32 [B*H*S] each;
+// acc_f32 != 0: dq / dk / dv are fp32 accumulators the gradients are added to
 int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, float* ws_delta, float* ws_lse2, unsigned* err, cudaStream_t stream);
+                  void* dv, float* ws_delta, float* ws_lse2, int acc_f32, unsigned* err,
+                  cudaStream_t stream);
 bool tc_fwd_supported(const AttnShape& sh);
 bool tc_bwd_supported(const AttnShape& sh);
 
@@ -94,5 +98,16 @@ enum KernelId : int {
 };
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);
+
+// An NVTX range named after the entry point, open for the duration of one C
+// ABI call (host side: argument checks and enqueueing), so that a timeline
+// profiler can attribute each kernel and copy to the call that issued it.
+// Without an attached tool the push / pop are no-ops.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 }  // namespace cpattn

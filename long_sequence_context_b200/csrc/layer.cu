@@ -232,6 +232,7 @@ int cpattn_layer_fwd(const void* x, const void* w_qkv, const void* b_qkv, const 
                      const void* b_o, void* y, void* q, void* k, void* v, void* o, float* lse,
                      int B, int S, int E, int H, int cp_size, int causal, float scale,
                      void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nv("cpattn_layer_fwd");
   int st = check_layer(B, S, E, H, cp_size, causal, scale);
   if (st != CPATTN_OK) return st;
   if (!x || !w_qkv || !b_qkv || !w_o || !b_o || !y || !q || !k || !v || !o || !lse) return CPATTN_ERR_ARG;
@@ -265,6 +266,7 @@ int cpattn_layer_bwd(const void* x, const void* w_qkv, const void* w_o, const vo
                      void* dw_qkv, void* db_qkv, void* dw_o, void* db_o, int B, int S, int E, int H,
                      int cp_size, int causal, float scale, void* workspace, size_t ws_bytes,
                      void* stream) {
+  NvtxRange nv("cpattn_layer_bwd");
   int st = check_layer(B, S, E, H, cp_size, causal, scale);
   if (st != CPATTN_OK) return st;
   if (!x || !w_qkv || !w_o || !q || !k || !v || !o || !lse || !dy || !dx || !dw_qkv || !db_qkv ||

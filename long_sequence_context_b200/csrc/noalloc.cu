@@ -8,8 +8,9 @@
 // callers can pass their inputs and outputs but cannot hand cpattn_bwd a
 // workspace.
 //
-// What it does: the backward's scratch (fp32 dQ accumulator and per-row delta)
-// lives in one fixed array in device global memory, declared below.  The
+// What it does: the backward's scratch -- two fp32 values per row, delta_i =
+// dO_i . O_i and LSE_i * log2(e) -- lives in one fixed array in device global
+// memory, declared below.  The
 // driver creates it when this library's module is loaded on a device, and
 // every device that loads the library keeps it until the process exits.  This
 // file never calls cudaMalloc, cudaFree or any allocating routine; it looks up
@@ -33,7 +34,9 @@ std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
 // Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does this set-up).
+// per device (the first call on a device does this set-up) and kept for the
+// process: the address belongs to the device's primary context, so the
+// library is not used across a cudaDeviceReset.
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CPATTN_ERR_CUDA;
@@ -60,8 +63,9 @@ extern "C" int cpattn_bwd_noalloc(const void* q, const void* k, const void* v, c
   void* scratch = nullptr;
   const int st = scratch_address(&scratch);
   if (st != CPATTN_OK) return st;
-  // cpattn_bwd treats its workspace as uninitialised and clears what it
-  // accumulates into, so the previous call's leftovers do not matter.
+  // cpattn_bwd treats its workspace as uninitialised: its preprocess kernel
+  // writes delta and LSE * log2(e) for every row of this call before the
+  // gradient kernels read them, so the previous call's leftovers are never used.
   return cpattn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, S, D, cp_size, causal, scale,
                     scratch, (size_t)CPATTN_NOALLOC_SCRATCH_BYTES, dtype, stream);
 }

@@ -60,6 +60,17 @@ __global__ void delta_kernel(const T* __restrict__ o, const T* __restrict__ dout
   if (lane == 0) delta[row] = acc;
 }
 
+// Output of one gradient element: written in the tensor's dtype, or, in
+// accumulate mode (acc != nullptr), added to the fp32 accumulator.  Each
+// element belongs to one thread of the launch.
+template <typename T>
+__device__ __forceinline__ void out_f(T* p, float* acc, long i, float x) {
+  if (acc)
+    acc[i] += x;
+  else
+    st_f(p, i, x);
+}
+
 constexpr int kTile = 16;   // keys (dK/dV kernel) or rows (dQ kernel) per block
 constexpr int kBatch = 8;   // rows / keys staged in shared memory at a time
 
@@ -71,6 +82,8 @@ __global__ void __launch_bounds__(128) dkdv_kernel(const T* __restrict__ q, cons
                                                    const T* __restrict__ dout,
                                                    const float* __restrict__ delta,
                                                    T* __restrict__ dk, T* __restrict__ dv,
+                                                   float* __restrict__ dk_acc_out,
+                                                   float* __restrict__ dv_acc_out,
                                                    RingGeom g, float scale) {
   constexpr int SL = D / 8;
   __shared__ float Qs[kBatch][D], dOs[kBatch][D], Ls[kBatch], Ds[kBatch];
@@ -137,8 +150,8 @@ __global__ void __launch_bounds__(128) dkdv_kernel(const T* __restrict__ q, cons
   }
 #pragma unroll
   for (int i = 0; i < SL; ++i) {
-    st_f(dk, base + (long)key * D + sl * SL + i, dk_acc[i] * scale);
-    st_f(dv, base + (long)key * D + sl * SL + i, dv_acc[i]);
+    out_f(dk, dk_acc_out, base + (long)key * D + sl * SL + i, dk_acc[i] * scale);
+    out_f(dv, dv_acc_out, base + (long)key * D + sl * SL + i, dv_acc[i]);
   }
 }
 
@@ -149,7 +162,8 @@ __global__ void __launch_bounds__(128) dq_kernel(const T* __restrict__ q, const 
                                                  const float* __restrict__ lse,
                                                  const T* __restrict__ dout,
                                                  const float* __restrict__ delta,
-                                                 T* __restrict__ dq, RingGeom g, float scale) {
+                                                 T* __restrict__ dq, float* __restrict__ dq_acc_out,
+                                                 RingGeom g, float scale) {
   constexpr int SL = D / 8;
   __shared__ float Ks[kBatch][D], Vs[kBatch][D];
   const long bh = blockIdx.y;
@@ -207,13 +221,13 @@ __global__ void __launch_bounds__(128) dq_kernel(const T* __restrict__ q, const 
     }
   }
 #pragma unroll
-  for (int i = 0; i < SL; ++i) st_f(dq, base + (long)row * D + sl * SL + i, acc[i] * scale);
+  for (int i = 0; i < SL; ++i) out_f(dq, dq_acc_out, base + (long)row * D + sl * SL + i, acc[i] * scale);
 }
 
 template <typename T, int D>
 int run_bwd(const AttnShape& sh, const void* q, const void* k, const void* v, const void* o,
             const float* lse, const void* dout, void* dq, void* dk, void* dv, float* ws_delta,
-            cudaStream_t stream) {
+            int acc_f32, cudaStream_t stream) {
   const long rows = (long)sh.B * sh.H * sh.S;
   const T* Q = static_cast<const T*>(q);
   const T* K = static_cast<const T*>(k);
@@ -226,13 +240,19 @@ int run_bwd(const AttnShape& sh, const void* q, const void* k, const void* v, co
   if (cudaGetLastError() != cudaSuccess) return -1;
   dim3 grid(sh.S / kTile, sh.B * sh.H);
   prof_begin(kKSimtDkdv, stream);
-  dkdv_kernel<T, D><<<grid, 128, 0, stream>>>(Q, K, V, lse, dO, ws_delta, static_cast<T*>(dk),
-                                              static_cast<T*>(dv), sh.g, sh.scale);
+  float* acc_dk = acc_f32 ? static_cast<float*>(dk) : nullptr;
+  float* acc_dv = acc_f32 ? static_cast<float*>(dv) : nullptr;
+  float* acc_dq = acc_f32 ? static_cast<float*>(dq) : nullptr;
+  dkdv_kernel<T, D><<<grid, 128, 0, stream>>>(Q, K, V, lse, dO, ws_delta,
+                                              acc_f32 ? nullptr : static_cast<T*>(dk),
+                                              acc_f32 ? nullptr : static_cast<T*>(dv), acc_dk,
+                                              acc_dv, sh.g, sh.scale);
   prof_end(kKSimtDkdv, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
   prof_begin(kKSimtDq, stream);
-  dq_kernel<T, D><<<grid, 128, 0, stream>>>(Q, K, V, lse, dO, ws_delta, static_cast<T*>(dq),
-                                            sh.g, sh.scale);
+  dq_kernel<T, D><<<grid, 128, 0, stream>>>(Q, K, V, lse, dO, ws_delta,
+                                            acc_f32 ? nullptr : static_cast<T*>(dq), acc_dq, sh.g,
+                                            sh.scale);
   prof_end(kKSimtDq, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
   return 3;
@@ -242,14 +262,17 @@ int run_bwd(const AttnShape& sh, const void* q, const void* k, const void* v, co
 
 int launch_simt_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                     const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                    void* dv, float* ws_delta, cudaStream_t stream) {
+                    void* dv, float* ws_delta, int acc_f32, cudaStream_t stream) {
   if (sh.bf16) {
     if (sh.D == 64)
-      return run_bwd<__nv_bfloat16, 64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, stream);
-    return run_bwd<__nv_bfloat16, 128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, stream);
+      return run_bwd<__nv_bfloat16, 64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, acc_f32,
+                                        stream);
+    return run_bwd<__nv_bfloat16, 128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, acc_f32,
+                                       stream);
   }
-  if (sh.D == 64) return run_bwd<float, 64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, stream);
-  return run_bwd<float, 128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, stream);
+  if (sh.D == 64)
+    return run_bwd<float, 64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, acc_f32, stream);
+  return run_bwd<float, 128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, acc_f32, stream);
 }
 
 }  // namespace cpattn

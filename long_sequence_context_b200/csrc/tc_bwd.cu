@@ -230,10 +230,16 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t ov[32];
         tmem_ld32<0>(tmem_base + lane_off + C::kColDV + col, ov);
         tmem_wait_ld();
-        store_row32(P.dv + orow + col, ov, 1.f);
+        if (P.acc_f32)
+          add_row32(P.dv_acc + orow + col, ov, 1.f);
+        else
+          store_row32(P.dv + orow + col, ov, 1.f);
         tmem_ld32<0>(tmem_base + lane_off + C::kColDK + col, ov);
         tmem_wait_ld();
-        store_row32(P.dk + orow + col, ov, P.scale);
+        if (P.acc_f32)
+          add_row32(P.dk_acc + orow + col, ov, P.scale);
+        else
+          store_row32(P.dk + orow + col, ov, P.scale);
       }
       tc_fence_before();
       mbar_arrive(acc_free);
@@ -445,7 +451,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
 template <int D>
 int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v, const void* o,
                 const float* lse, const void* dout, void* dq, void* dk, void* dv, float* ws_delta,
-                float* ws_lse2, unsigned* err, cudaStream_t stream) {
+                float* ws_lse2, int acc_f32, unsigned* err, cudaStream_t stream) {
   const long rows = (long)sh.B * sh.H * sh.S;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_tmap_bf16_2d(&mq, q, rows, D, 64, 128) || !make_tmap_bf16_2d(&mk, k, rows, D, 64, 128) ||
@@ -474,6 +480,10 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.dq = static_cast<__nv_bfloat16*>(dq);
   P.dk = static_cast<__nv_bfloat16*>(dk);
   P.dv = static_cast<__nv_bfloat16*>(dv);
+  P.acc_f32 = acc_f32;
+  P.dq_acc = static_cast<float*>(dq);
+  P.dk_acc = static_cast<float*>(dk);
+  P.dv_acc = static_cast<float*>(dv);
   P.err = err;
   static std::atomic<unsigned long long> attr_done{0};
   if (!smem_attr_once(tc_dkdv_kernel<D>, DkdvCfg<D>::kSmemBytes, attr_done)) return -1;
@@ -502,10 +512,13 @@ bool tc_bwd_supported(const AttnShape& sh) {
 
 int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void* v,
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
-                  void* dv, float* ws_delta, float* ws_lse2, unsigned* err, cudaStream_t stream) {
+                  void* dv, float* ws_delta, float* ws_lse2, int acc_f32, unsigned* err,
+                  cudaStream_t stream) {
   if (sh.D == 64)
-    return bwd::launch_impl<64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
-  return bwd::launch_impl<128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, err, stream);
+    return bwd::launch_impl<64>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, acc_f32,
+                                err, stream);
+  return bwd::launch_impl<128>(sh, q, k, v, o, lse, dout, dq, dk, dv, ws_delta, ws_lse2, acc_f32,
+                               err, stream);
 }
 
 }  // namespace cpattn

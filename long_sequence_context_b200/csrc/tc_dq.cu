@@ -6,7 +6,8 @@
 //   P_j  = exp2(S_j * scale * log2 e - LSE * log2 e)   (DIAG tiles masked)
 //   dS_j = P_j (dP_j - delta)                          (bf16, back into TMEM)
 //   dQ  += dS_j K_j                                    (A = dS_j from TMEM)
-// dQ accumulates in TMEM and is written once, scaled, as bf16: no reductions.
+// dQ accumulates in TMEM and is written once, scaled, as bf16 (in accumulate
+// mode: added once into the caller's fp32 dQ sum): no reductions.
 //
 // Overlap.  S is double-buffered; the elementwise work of a tile is split into
 // an exponential phase that needs only S_j and a dS phase that needs dP_j.  The
@@ -188,7 +189,10 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t v[32];
         tmem_ld32<0>(tmem_base + lane_off + C::kColDQ + col, v);
         tmem_wait_ld();
-        store_row32(P.dq + row * D + col, v, P.scale);
+        if (P.acc_f32)
+          add_row32(P.dq_acc + row * D + col, v, P.scale);
+        else
+          store_row32(P.dq + row * D + col, v, P.scale);
       }
       tc_fence_before();
       mbar_arrive(acc_free);

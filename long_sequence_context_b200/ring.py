@@ -19,9 +19,10 @@ schedules the blocks and moves chunks between ranks:
 
     forward   per block  cpattn_fwd_step on the (q chunk, kv chunk) pair
               per row    cpattn_merge of the block partials, cpattn_finalize
-    backward  per block  cpattn_bwd on the pair with the rows' final O and LSE
-                         (its exp(s - LSE) and dO.O are those of the whole row)
-              sums       cpattn_accumulate into fp32 dQ, dK, dV
+    backward  per block  cpattn_bwd_accumulate on the pair with the rows' final
+                         O and LSE (its exp(s - LSE) and dO.O are those of the
+                         whole row), adding the block's terms in fp32 to the
+                         running dQ, dK, dV sums (one rounding, at the end)
 
 The schedule is written once, as a generator that yields its exchanges
 ("start" a send to rank + 1 / receive from rank - 1, "finish" it); run_dist
@@ -80,15 +81,14 @@ class CudaBlocks:
     def zeros_f32(self, like):
         return torch.zeros(like.shape, dtype=torch.float32, device=like.device)
 
-    def bwd(self, q, k, v, o, lse, do, diag: bool):
+    def bwd_into(self, q, k, v, o, lse, do, diag: bool, dq_acc, dk_acc, dv_acc):
+        """Adds the block's dQ, dK, dV terms, in fp32, to the three sums."""
         B, H, S, D = q.shape
         need = self.cp.bwd_workspace_bytes(B, H, S, D)
         if self._ws is None or self._ws.numel() < need:
             self._ws = torch.empty(need, dtype=torch.uint8, device=q.device)
-        return self.cp.bwd(q, k, v, o, lse, do, 1, causal=diag, scale=self.scale, workspace=self._ws)
-
-    def accumulate(self, acc, x):
-        self.cp.accumulate_(acc, x)
+        self.cp.bwd_accumulate_(q, k, v, o, lse, do, dq_acc, dk_acc, dv_acc, 1, causal=diag,
+                                scale=self.scale, workspace=self._ws)
 
     def cast(self, acc, dtype):
         return self.cp.finalize(acc, dtype)
@@ -138,10 +138,8 @@ def bwd_schedule(rank, world, q, k, v, o, lse, do, causal, be):
                 kind = block_kind(a, b, causal)
                 if kind == SKIP:
                     continue
-                gq, gk, gv = be.bwd(q[ai], kv[bi], kv[n + bi], o[ai], lse[ai], do[ai], kind == DIAG)
-                be.accumulate(dq[ai], gq)
-                be.accumulate(dkv[bi], gk)
-                be.accumulate(dkv[n + bi], gv)
+                be.bwd_into(q[ai], kv[bi], kv[n + bi], o[ai], lse[ai], do[ai], kind == DIAG,
+                            dq[ai], dkv[bi], dkv[n + bi])
         if world > 1:
             # the sums travel with their K/V; after the last step they reach
             # the chunks' owner

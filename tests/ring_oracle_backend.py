@@ -42,6 +42,12 @@ class OracleBlocks:
     def zeros_f32(self, like):
         return torch.zeros(like.shape, dtype=torch.float64)
 
+    def bwd_into(self, q, k, v, o, lse, do, diag, dq_acc, dk_acc, dv_acc):
+        dq, dk, dv = self.bwd(q, k, v, o, lse, do, diag)
+        dq_acc += dq
+        dk_acc += dk
+        dv_acc += dv
+
     def bwd(self, q, k, v, o, lse, do, diag):
         s = self.scale * torch.einsum("bhid,bhjd->bhij", q, k)
         p = torch.exp(s - lse[..., None])
@@ -55,9 +61,6 @@ class OracleBlocks:
         dq = self.scale * torch.einsum("bhij,bhjd->bhid", ds, k)
         dk = self.scale * torch.einsum("bhij,bhid->bhjd", ds, q)
         return dq, dk, dv
-
-    def accumulate(self, acc, x):
-        acc += x
 
     def cast(self, acc, dtype):
         return acc.clone()

@@ -63,14 +63,28 @@ FULL = ["causal_b1h32s32768d128_cp8_bf16", "noncausal_b2h32s16384d128_cp2_bf16",
         "causal_b1h8s131072d128_cp16_bf16"]
 
 
+def early_and_late_keys(S, n_chunks, seed):
+    """Key columns whose dK / dV sum over long ring walks: the first key of
+    every chunk and 16 seeded keys from the first half of the sequence (every
+    query row after them sees them, so their terms come from q tiles of every
+    virtual rank at every ring step), plus the last 32 keys (a DIAG corner)."""
+    c = S // n_chunks
+    g = np.random.default_rng(1000 + seed)
+    cols = {a * c for a in range(n_chunks)}
+    cols |= {int(x) for x in g.integers(0, S // 2, size=16)}
+    cols |= set(range(S - 32, S))
+    return np.array(sorted(cols), dtype=np.int64)
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_bwd_full_workload_sampled(cp, name):
     w = WORKLOADS[name]
     q, k, v, dout = workload_inputs(w)
     dq, dk, dv = run_fwd_bwd(cp, q, k, v, dout, w.cp_size, w.causal)
     n_chunks = 2 * w.cp_size if w.causal else w.cp_size
-    # dQ on sampled rows of two heads; dK / dV on the last 32 key columns of one
-    # head (rows that see them are few when causal; all rows otherwise)
+    # dQ on sampled rows of two heads; dK / dV of one head on early keys (long
+    # walks over every ring step) and the last 32 keys when causal, on four keys
+    # (each seen by every row) otherwise
     for b, h in ((0, 0), (w.B - 1, w.H - 1)):
         sl = (slice(b, b + 1), slice(h, h + 1))
         args = [np64(t[sl]) for t in (q, k, v, dout)]
@@ -80,7 +94,7 @@ def test_bwd_full_workload_sampled(cp, name):
     b, h = 0, w.H // 2
     sl = (slice(b, b + 1), slice(h, h + 1))
     args = [np64(t[sl]) for t in (q, k, v, dout)]
-    cols = np.arange(w.S - 32, w.S) if w.causal else np.array([0, 1, w.S // 2, w.S - 1])
+    cols = early_and_late_keys(w.S, n_chunks, seed=h) if w.causal else np.array([0, 1, w.S // 2, w.S - 1])
     rk, rv = orc.attn_bwd_kv_cols(*args, w.causal, w.scale, 0, 0, cols)
     assert_close(dk[b, h, cols], rk, torch.bfloat16, f"{name} dK cols")
     assert_close(dv[b, h, cols], rv, torch.bfloat16, f"{name} dV cols")
@@ -91,3 +105,57 @@ def test_bwd_full_workload_sampled(cp, name):
     dk_abs = np.abs(np64(dk)).sum(axis=2)
     assert np.all(np.abs(dk_sum) <= 1e-2 * dk_abs + 1e-2), float(np.max(np.abs(dk_sum)))
     assert np.max(np.abs(dv_sum - do_sum)) <= 1e-2 * w.S ** 0.5, float(np.max(np.abs(dv_sum - do_sum)))
+
+
+ACC_CASES = [
+    (1, 2, 1024, 128, 2, True, torch.bfloat16, 0),   # tcgen05 kernels
+    (1, 2, 1024, 64, 2, False, torch.bfloat16, 0),
+    (1, 2, 1024, 128, 4, True, torch.bfloat16, 1),   # CUDA-core kernels
+    (1, 2, 256, 64, 2, True, torch.float32, 0),      # fp32: CUDA-core kernels (automatic)
+]
+
+
+@pytest.mark.parametrize("B,H,S,D,cp_size,causal,dtype,path", ACC_CASES)
+def test_bwd_accumulate_adds_the_gradients_in_fp32(cp, B, H, S, D, cp_size, causal, dtype, path):
+    """cpattn_bwd_accumulate adds dQ, dK, dV into fp32 sums: from zero, one
+    rounding of the sum gives cpattn_bwd's output exactly; from a seeded start,
+    two calls add twice the gradient (checked against the oracle)."""
+    q, k, v, dout = make_qkv(B, H, S, D, dtype, seed=300 + S + D + path)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    prev = cp.set_path(path)
+    try:
+        o, lse = cp.fwd(qd, kd, vd, cp_size, causal)
+        ref = cp.bwd(qd, kd, vd, o, lse, dod, cp_size, causal)
+        zero = [torch.zeros(q.shape, dtype=torch.float32, device="cuda") for _ in range(3)]
+        cp.bwd_accumulate_(qd, kd, vd, o, lse, dod, *zero, cp_size, causal)
+        gen = torch.Generator().manual_seed(7)
+        start = [torch.randn(q.shape, generator=gen, dtype=torch.float32) for _ in range(3)]
+        acc = [t.cuda() for t in start]
+        cp.bwd_accumulate_(qd, kd, vd, o, lse, dod, *acc, cp_size, causal)
+        cp.bwd_accumulate_(qd, kd, vd, o, lse, dod, *acc, cp_size, causal)
+        assert cp.sync_status() == cp.OK
+        assert cp.last_path() == (1 if dtype == torch.float32 else path)
+    finally:
+        cp.set_path(prev)
+    for name, z, r in zip(("dQ", "dK", "dV"), zero, ref):
+        assert torch.equal(z.to(dtype), r), f"{name}: one rounding of the fp32 sum differs from cpattn_bwd"
+    want = orc.attn_bwd(np64(q), np64(k), np64(v), np64(dout), causal, D ** -0.5)
+    for name, a, s0, w_ in zip(("dQ", "dK", "dV"), acc, start, want):
+        got = (np64(a.cpu()) - np64(s0)) / 2.0
+        assert_close(got, w_, dtype, f"{name} (two accumulating calls)")
+
+
+def test_bwd_accumulate_rejects_mismatched_accumulators(cp):
+    q = torch.zeros((1, 1, 256, 64), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 1, 256), dtype=torch.float32, device="cuda")
+    good = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
+    bf = torch.zeros(q.shape, dtype=torch.bfloat16, device="cuda")
+    short = torch.zeros((1, 1, 128, 64), dtype=torch.float32, device="cuda")
+    n0 = cp.launch_count()
+    with pytest.raises(TypeError):
+        cp.bwd_accumulate_(q, q, q, q, lse, q, bf, good, good.clone(), 1, True)
+    with pytest.raises(ValueError):
+        cp.bwd_accumulate_(q, q, q, q, lse, q, good, short, good.clone(), 1, True)
+    with pytest.raises(ValueError):
+        cp.bwd_accumulate_(q, q, q, q, lse, q, good, good, good.clone(), 1, True)
+    assert cp.launch_count() == n0

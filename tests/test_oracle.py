@@ -314,11 +314,43 @@ def test_plan_noncausal_contiguous():
     assert sorted((a, b) for _, _, a, b, _, _ in rows) == [(a, b) for a in range(4) for b in range(4)]
 
 
-def test_planted_ring_mistake_is_caught():
-    # a plan that reads (r + t) instead of (r - t) still covers every block
-    # once, but then a wrong DIAG/FULL labelling must be caught by the exact
-    # cover check; here we plant a dropped-block mistake and verify detection
-    rows = [r for r in oplan.plan_rows(32, 4, True) if not (r[2] == 5 and r[3] == 2)]
-    covered = {(a, b) for _, _, a, b, _, kind in rows if kind != oplan.SKIP}
-    assert (5, 2) not in covered
-    assert covered != {(a, b) for a in range(8) for b in range(8) if a >= b}
+def _plan_pins_fail(monkeypatch, **planted):
+    """True when at least one of the plan pins above fails with `planted`
+    functions swapped into the plan oracle (on the CPU, for this test only)."""
+    for name, fn in planted.items():
+        monkeypatch.setattr(oplan, name, fn)
+    checks = [test_plan_golden_zigzag_cp4, test_plan_noncausal_contiguous] + \
+             [lambda cp=cp: test_plan_invariants(cp) for cp in (1, 2, 3, 4, 8, 16)]
+    failed = 0
+    for check in checks:
+        try:
+            check()
+        except AssertionError:
+            failed += 1
+    return failed > 0
+
+
+@pytest.mark.parametrize("mistake", ["zigzag_off_by_one", "contiguous_when_causal", "diag_as_full",
+                                     "ring_reads_ahead", "skip_as_full"])
+def test_plan_pins_catch_planted_mistakes(monkeypatch, mistake):
+    """Plausible mistakes planted in the plan oracle: each must make at least
+    one of the plan pins (golden example, invariants) fail."""
+    own, kind, rows = oplan.owned_chunks, oplan.block_kind, oplan.plan_rows
+    if mistake == "zigzag_off_by_one":       # rank r owns {r, 2N-2-r}
+        planted = {"owned_chunks": lambda r, n, c: [r, 2 * n - 2 - r] if c else [r]}
+    elif mistake == "contiguous_when_causal":  # rank r owns {2r, 2r+1}
+        planted = {"owned_chunks": lambda r, n, c: [2 * r, 2 * r + 1] if c else [r]}
+    elif mistake == "diag_as_full":          # the diagonal block left unmasked
+        planted = {"block_kind": lambda a, b, c: oplan.FULL if (c and a == b) else kind(a, b, c)}
+    elif mistake == "skip_as_full":          # a future block computed
+        planted = {"block_kind": lambda a, b, c: oplan.FULL if c else kind(a, b, c)}
+    else:                                    # step t reads rank (r + t) mod N, src field kept
+        def ahead(S, n, c):
+            out = []
+            for r, t, a, b, src, k in rows(S, n, c):
+                s2 = (r + t) % n
+                b2 = own(s2, n, c)[own(src, n, c).index(b)]
+                out.append((r, t, a, b2, src, kind(a, b2, c)))
+            return out
+        planted = {"plan_rows": ahead}
+    assert _plan_pins_fail(monkeypatch, **planted)

@@ -43,6 +43,8 @@ def test_noalloc_matches_workspace_backward_twice(cp, B, H, S, D, cp_size, causa
         assert cp.sync_status() == cp.OK
         for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
             assert_close(g.cpu(), np64(r.cpu()), dtype, f"call {call} {name}")
+            # same kernels, same inputs, no atomics: the results are identical
+            assert torch.equal(g, r), f"call {call} {name}: differs from cpattn_bwd"
 
 
 def test_noalloc_rejects_shapes_beyond_the_scratch(cp):

@@ -51,20 +51,3 @@ def sample_rows(S, n_chunks, n_total=128, seed=0):
     while len(rows) < min(n_total, S):
         rows.add(int(g.integers(S)))
     return np.array(sorted(rows), dtype=np.int64)
-
-
-def assert_close_block_sum(got, want, n_terms, what=""):
-    """Bar for a gradient summed (in fp32) from n_terms block terms that the
-    library's backward returns rounded to bf16 (the multi-rank paths): each
-    term carries up to half a bf16 ulp (2^-9 relative), so the max-abs bar is
-    the bf16 bar plus n_terms * 2^-9 * max|want|; the mean-abs bar is unchanged."""
-    got = np64(got) if isinstance(got, torch.Tensor) else np.asarray(got, dtype=np.float64)
-    want = np.asarray(want, dtype=np.float64)
-    assert got.shape == want.shape, (what, got.shape, want.shape)
-    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
-    err = np.abs(got - want)
-    bar = BF16_MAX + n_terms * 2.0 ** -9 * float(np.abs(want).max(initial=0.0))
-    mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
-    assert mx <= bar and mean <= BF16_MEAN, \
-        f"{what}: max-abs {mx:.3e} (bar {bar:.3e}), mean-abs {mean:.3e} (bar {BF16_MEAN})"
-    return mx, mean
