@@ -659,6 +659,17 @@ def run_layer(args, w):
         ach = heads_bytes / (hk["ms_total"] / args.steps * 1e-3) / 1e9
         heads_roof = {"bound": "hbm", "kernel": "layer_heads", "achieved": ach, "peak": peaks["hbm_gbs"],
                       "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    # projection GEMMs (tensor-bound): 8*B*S*E^2 FLOPs forward, twice that backward
+    gk = per_kernel.get("gemm")
+    gemm_roof = None
+    if gk:
+        g_flops = 24.0 * B * S * E * E
+        g_ms = gk["ms_total"] / args.steps
+        ach = g_flops / (g_ms * 1e-3) / 1e12
+        gemm_roof = {"bound": "tensor", "kernel": "gemm", "ms_per_step": g_ms, "launches_per_step":
+                     gk["launches"] / args.steps, "achieved": ach, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                     "peak_kind": f"bf16_tflops ({peaks['source']})"}
     if rank == 0:
         line = {
             "metric": LAYER_METRIC, "value": (f_fwd + f_bwd) * world / (ms_step * 1e-3) / 1e12,
@@ -669,7 +680,8 @@ def run_layer(args, w):
                        "cp_size": w.cp_size, "causal": w.causal},
             "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd},
             "per_kernel_ms": per_kernel,
-            "cublaslt_gemm_ms_per_step": ms_step - own_ms,
+            "gemm_roofline": gemm_roof,
+            "unattributed_ms_per_step": ms_step - own_ms,
             "heads_roofline": heads_roof,
             "gpu_launches": launches,
             "clocks": clk,

@@ -241,13 +241,14 @@ int cpattn_accumulate(float* acc, const void* x, long n, int dtype, void* stream
  *     w_o, dw_o              [E][E];   b_o, db_o [E]
  *     q, k, v, o             [B][H][S][D] (bf16), lse [B][H][S] (fp32): saved
  *                                      by the forward for the backward
- *   The projections run on cuBLASLt (bf16, fp32 accumulation, the bias added
- *   in the GEMM epilogue) with the caller's workspace; the head reshapes and
- *   the bias gradients are this library's kernels.
+ *   The projections run on this library's tcgen05 GEMM (cpattn_gemm below:
+ *   bf16, fp32 accumulation, the bias added in the GEMM epilogue); the head
+ *   reshapes and the bias gradients are this library's kernels too.  B*S and E
+ *   must be multiples of 8 (CPATTN_ERR_SHAPE).
  *   Workspace: cpattn_layer_workspace_bytes(B, S, E, H) bytes (0 for invalid
  *   sizes), used by both calls; its contents need not survive between them.
  *   Errors: CPATTN_ERR_SHAPE / ARG / ALIGN / WORKSPACE before anything is
- *   enqueued; CPATTN_ERR_CUDA when a launch or a cuBLASLt call fails.
+ *   enqueued; CPATTN_ERR_CUDA when a launch fails.
  */
 size_t cpattn_layer_workspace_bytes(int B, int S, int E, int H);
 
@@ -266,6 +267,24 @@ int cpattn_layer_bwd(const void* x, const void* w_qkv, const void* w_o, const vo
                      const void* dy, void* dx, void* dw_qkv, void* db_qkv, void* dw_o,
                      void* db_o, int B, int S, int E, int H, int cp_size, int causal,
                      float scale, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * cpattn_gemm -- the layer's projection GEMM on the tcgen05 tensor cores:
+ *     C[M][N] = op(A) op(B) (+ bias[n] added to every row),
+ * bf16 operands, bias and result (round to nearest even), fp32 accumulation,
+ * all row-major and caller-owned device memory.  The products of the
+ * attention layer's nn.Linear projections and their gradients ("Configuring
+ * RingAttention+FlashAttention for CP", section 3 code: q/k/v_proj, out_proj).
+ *   a_layout 0: A stored [M][K];   1: A stored [K][M] (A is its transpose)
+ *   b_layout 0: B stored [N][K] (the nn.Linear weight layout, C = A B^T);
+ *            1: B stored [K][N] (C = A B)
+ *   bias: [N] or NULL.  C must not alias A, B or bias.
+ *   M, N, K >= 1 and multiples of 8 (CPATTN_ERR_SHAPE); pointers 16-byte
+ *   aligned (CPATTN_ERR_ALIGN); layouts other than 0 / 1: CPATTN_ERR_ARG.
+ *   In-kernel bounded-wait failures are reported by cpattn_sync_status().
+ */
+int cpattn_gemm(const void* A, const void* B, const void* bias, void* C, int M, int N, int K,
+                int a_layout, int b_layout, void* stream);
 
 /*
  * cpattn_sync_status -- synchronises `stream`, then returns and clears the
@@ -303,9 +322,9 @@ long long cpattn_launch_count(void);
  *   since the last cpattn_profile(1); waits for those events.  Kernel kinds:
  *   0 tcgen05 forward, 1 CUDA-core forward, 2 merge, 3 finalize, 4 backward
  *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 dK/dV,
- *   8 tcgen05 dQ, 9 layer head split / merge, 10 layer bias gradients (the
- *   layer's cuBLASLt GEMMs are not this library's kernels and are not timed),
- *   11 gradient accumulation (cpattn_accumulate).
+ *   8 tcgen05 dQ, 9 layer head split / merge, 10 layer bias gradients,
+ *   11 gradient accumulation (cpattn_accumulate), 12 GEMM (cpattn_gemm and
+ *   the layer's projections).
  */
 int cpattn_profile(int on);
 int cpattn_profile_read(int kernel_kind, double* total_ms, long long* launches);

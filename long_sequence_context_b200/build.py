@@ -4,8 +4,8 @@
 
 Each csrc/*.cu is compiled by nvcc (-gencode arch=compute_100a,code=sm_100a
 -O3 -lineinfo) into _build/, then linked into long_sequence_context_b200/
-libcpattn.so with the CUDA runtime linked statically and cuBLASLt (used by the
-attention layer's projections) linked dynamically.
+libcpattn.so with the CUDA runtime linked statically.  No vendor math library
+is linked: every kernel is this package's own.
 """
 import concurrent.futures as cf
 import glob
@@ -65,7 +65,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if todo or _stale(LIB, objs):
         cuda_lib = os.path.join(os.path.dirname(os.path.dirname(NVCC)), "lib64")
         cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
-               "-o", LIB] + objs + ["-L" + cuda_lib, "-lcublasLt", "-Xlinker", "-rpath," + cuda_lib]
+               "-o", LIB] + objs + ["-L" + cuda_lib, "-Xlinker", "-rpath," + cuda_lib]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -25,7 +25,7 @@ EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpat
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
            "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc",
            "cpattn_layer_workspace_bytes", "cpattn_layer_fwd", "cpattn_layer_bwd",
-           "cpattn_accumulate", "cpattn_bwd_accumulate"]
+           "cpattn_accumulate", "cpattn_bwd_accumulate", "cpattn_gemm"]
 
 # size of the library's fixed scratch array behind bwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -64,6 +64,7 @@ def _load():
         "cpattn_layer_workspace_bytes": ([i, i, i, i], sz),
         "cpattn_accumulate": ([vp, vp, l, i, vp], i),
         "cpattn_layer_fwd": ([vp] * 11 + [i] * 6 + [f, vp, sz, vp], i),
+        "cpattn_gemm": ([vp, vp, vp, vp, i, i, i, i, i, vp], i),
         "cpattn_layer_bwd": ([vp] * 14 + [i] * 6 + [f, vp, sz, vp], i),
     }
     for name, (args, res) in sigs.items():
@@ -306,6 +307,31 @@ def accumulate_(acc, x, stream=None):
     return acc
 
 
+def gemm(a, b, bias=None, a_t: bool = False, b_t: bool = False, out=None, stream=None):
+    """C = op(a) op(b) (+ bias) on the library's tcgen05 GEMM, bf16, fp32 accumulation.
+    a: [M, K] (a_t: [K, M], used transposed); b: [N, K] as an nn.Linear weight
+    (C = a b^T), or with b_t: [K, N] (C = a b).  bias: [N] or None."""
+    for t, n in ((a, "a"), (b, "b")):
+        if not isinstance(t, torch.Tensor) or t.dim() != 2:
+            raise ValueError(f"{n} must be a 2-D tensor")
+    M, K = (a.shape[1], a.shape[0]) if a_t else (a.shape[0], a.shape[1])
+    N = b.shape[1] if b_t else b.shape[0]
+    kb = b.shape[0] if b_t else b.shape[1]
+    if kb != K:
+        raise ValueError(f"inner dimensions differ: a gives K={K}, b gives {kb}")
+    _expect(a, "a", a.shape, torch.bfloat16)
+    _expect(b, "b", b.shape, torch.bfloat16, a)
+    if bias is not None:
+        _expect(bias, "bias", (N,), torch.bfloat16, a)
+    if out is not None:
+        _expect(out, "out", (M, N), torch.bfloat16, a)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else out
+    _check(lib.cpattn_gemm(_dev(a, "a"), _dev(b, "b"),
+                           _dev(bias, "bias") if bias is not None else None, _dev(c, "out"),
+                           M, N, K, int(a_t), int(b_t), _stream(stream)), "cpattn_gemm")
+    return c
+
+
 def layer_workspace_bytes(B, S, E, H) -> int:
     return int(lib.cpattn_layer_workspace_bytes(B, S, E, H))
 
@@ -396,7 +422,7 @@ def debug_stall(n: int) -> int:
 
 KERNEL_KINDS = {0: "tc_fwd", 1: "simt_fwd", 2: "merge", 3: "finalize", 4: "bwd_delta",
                 5: "simt_dkdv", 6: "simt_dq", 7: "tc_dkdv", 8: "tc_dq", 9: "layer_heads",
-                10: "layer_colsum", 11: "accumulate"}
+                10: "layer_colsum", 11: "accumulate", 12: "gemm"}
 
 
 def profile(on: bool) -> int:

@@ -96,6 +96,8 @@ int check_attention_shape(int B, int H, int S, int D, int cp_size, int causal, f
 }
 
 void add_launches(int n) { g_launches += n; }
+
+unsigned* device_error_word() { return err_word(); }
 }  // namespace cpattn
 
 namespace {

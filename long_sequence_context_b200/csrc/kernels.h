@@ -56,6 +56,17 @@ bool tc_bwd_supported(const AttnShape& sh);
 
 int num_sms(int device);
 
+// Device address of the library's error word on the current device (looked up
+// once per device), or null when the lookup failed.
+unsigned* device_error_word();
+
+// ---- tcgen05 GEMM (gemm.cu): C[M][N] = op(A) op(B) (+ bias[N]), bf16, fp32 accumulation.
+// a_mn: A stored [K][M] (else [M][K]); b_mn: B stored [K][N] (else [N][K]).
+// gemm_check: 0 when the sizes are supported (M, N, K >= 1, multiples of 8).
+int gemm_check(int M, int N, int K);
+int launch_gemm(const void* A, const void* B, const void* bias, void* C, int M, int N, int K,
+                int a_mn, int b_mn, unsigned* err, cudaStream_t stream);
+
 // The attention entry points' shape and argument rules (CPATTN_OK or the
 // status cpattn_fwd / cpattn_bwd would return), for callers that compose them.
 int check_attention_shape(int B, int H, int S, int D, int cp_size, int causal, float scale,
@@ -94,7 +105,8 @@ enum KernelId : int {
   kKLayerHeads = 9,   // head split / merge of the attention layer
   kKLayerColsum = 10, // bias gradients of the attention layer
   kKAccumulate = 11,  // fp32 gradient sums of the multi-rank ring backward
-  kKNumKernels = 12
+  kKGemm = 12,        // projection GEMMs of the attention layer (cpattn_gemm)
+  kKNumKernels = 13
 };
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);

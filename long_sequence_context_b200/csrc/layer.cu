@@ -5,14 +5,11 @@
 // width E, q.view(B,S,H,D).transpose(1,2) before the ring loop, the inverse
 // transpose and out_proj after it.
 //
-// The projections are plain GEMMs and run on cuBLASLt (bf16 in/out, fp32
-// accumulate; the forward bias is fused as the GEMM epilogue).  The head
-// reshapes and the bias gradients are this library's own kernels; the
-// attention in between is cpattn_fwd / cpattn_bwd.
-//
-// Row-major matrices are handed to cuBLASLt as their column-major transposes:
-// Y[M,N] = X[M,K] W[N,K]^T is computed as Y^T = W X^T (m = N, n = M, k = K).
-#include <cublasLt.h>
+// The projections run on this library's tcgen05 GEMM (gemm.cu: bf16 in/out,
+// fp32 accumulate; the forward bias fused into its epilogue).  The head
+// reshapes and the bias gradients are this library's own kernels too; the
+// attention in between is cpattn_fwd / cpattn_bwd.  Nothing here calls a
+// vendor library.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -27,73 +24,18 @@
 namespace cpattn {
 namespace {
 
-constexpr size_t kLtWorkspace = 32u << 20;  // cuBLASLt workspace inside the layer workspace
-
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Per-device cuBLASLt handle, created on first use (host object only).
-cublasLtHandle_t lt_handle() {
-  static std::mutex mu;
-  static cublasLtHandle_t handles[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!handles[dev] && cublasLtCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
-  return handles[dev];
-}
-
-// Column-major C[m,n] = op(A) op(B) (+ bias[m] broadcast over n when bias != null),
-// bf16 operands and result, fp32 accumulation.  lda/ldb/ldc are column-major
-// leading dimensions of the stored (untransposed) matrices.
-bool gemm(cudaStream_t s, bool ta, bool tb, int m, int n, int k, const void* A, int lda,
-          const void* B, int ldb, void* C, int ldc, const void* bias, void* ws, float beta = 0.f) {
-  cublasLtHandle_t h = lt_handle();
-  if (!h) return false;
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  bool ok = false;
-  do {
-    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
-    const cublasOperation_t oa = ta ? CUBLAS_OP_T : CUBLAS_OP_N, ob = tb ? CUBLAS_OP_T : CUBLAS_OP_N;
-    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &oa, sizeof(oa));
-    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &ob, sizeof(ob));
-    if (bias) {
-      const cublasLtEpilogue_t epi = CUBLASLT_EPILOGUE_BIAS;
-      const cudaDataType_t bt = CUDA_R_16BF;
-      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_EPILOGUE, &epi, sizeof(epi));
-      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_BIAS_POINTER, &bias, sizeof(bias));
-      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_BIAS_DATA_TYPE, &bt, sizeof(bt));
-    }
-    if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, ta ? k : m, ta ? m : k, lda) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, tb ? n : k, tb ? k : n, ldb) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, m, n, ldc) != CUBLAS_STATUS_SUCCESS)
-      break;
-    if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
-    const size_t wsz = kLtWorkspace;
-    cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &wsz, sizeof(wsz));
-    cublasLtMatmulHeuristicResult_t res;
-    int found = 0;
-    if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &found) !=
-            CUBLAS_STATUS_SUCCESS ||
-        found < 1)
-      break;
-    const float alpha = 1.f;
-    ok = cublasLtMatmul(h, op, &alpha, A, la, B, lb, &beta, C, lc, C, lc, &res.algo, ws, wsz, s) ==
-         CUBLAS_STATUS_SUCCESS;
-  } while (false);
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return ok;
-}
-
-// Row-major Y[M,N] (+)= X[M,K] W[N,K]^T (+ bias[N])
-bool linear(cudaStream_t s, const void* X, const void* W, const void* bias, void* Y, int M, int N,
-            int K, void* ws) {
-  return gemm(s, true, false, N, M, K, W, K, X, K, Y, N, bias, ws);
+// Row-major C[M][N] = op(A) op(B) (+ bias[N]) on the tcgen05 GEMM.
+// a_mn: A stored [K][M]; b_mn: B stored [K][N] (otherwise [M][K] / [N][K]).
+bool gemm(cudaStream_t s, const void* A, const void* B, const void* bias, void* C, int M, int N,
+          int K, int a_mn, int b_mn) {
+  unsigned* err = device_error_word();
+  if (!err || gemm_check(M, N, K) != 0) return false;
+  const int n = launch_gemm(A, B, bias, C, M, N, K, a_mn, b_mn, err, s);
+  if (n < 0) return false;
+  add_launches(n);
+  return true;
 }
 
 // Head reshapes, 16 bytes (8 bf16) per thread.
@@ -178,12 +120,12 @@ bool colsum(cudaStream_t s, const void* Y, void* db, long rows, int N, float* pa
 }
 
 struct LayerWs {
-  size_t qkv, om, dom, dq, dk, dv, dout, attn, part, lt, total;
+  size_t qkv, om, dom, dq, dk, dv, dout, attn, part, total;
 };
 
 // Offsets of the layer workspace.  Forward: qkv [B*S][3E], om [B*S][E], lt.
 // Backward: om, dom [B*S][E], dout, dq, dk, dv [B][H][S][D], dqkv (reuses qkv),
-// the attention backward's workspace, the column-sum partials and lt.
+// the attention backward's workspace and the column-sum partials.
 LayerWs layer_ws(int B, int S, int E, int H) {
   const size_t rows = (size_t)B * S, t = rows * E * 2;
   LayerWs w;
@@ -197,7 +139,6 @@ LayerWs layer_ws(int B, int S, int E, int H) {
   w.dv = off;   off += align256(t);
   w.attn = off; off += align256(cpattn_bwd_workspace_bytes(B, H, S, E / H));
   w.part = off; off += align256((size_t)kColsumSplits * 3 * E * 4);
-  w.lt = off;   off += align256(kLtWorkspace);
   w.total = off;
   return w;
 }
@@ -208,6 +149,7 @@ int check_layer(int B, int S, int E, int H, int cp_size, int causal, float scale
   const int D = E / H;
   if (D != 64 && D != 128) return CPATTN_ERR_SHAPE;
   if ((long long)B * S * 3 * E >= (1LL << 31)) return CPATTN_ERR_SHAPE;  // GEMM dims and offsets
+  if ((B * S) % 8 != 0 || E % 8 != 0) return CPATTN_ERR_SHAPE;           // GEMM row alignment
   (void)cp_size;
   (void)causal;
   if (!(scale > 0.f) || !std::isfinite(scale)) return CPATTN_ERR_ARG;
@@ -249,15 +191,14 @@ int cpattn_layer_fwd(const void* x, const void* w_qkv, const void* b_qkv, const 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* qkv = ws + w.qkv;
   void* om = ws + w.om;
-  void* lt = ws + w.lt;
   const int rows = B * S;
   // q|k|v = x Wqkv^T + bqkv  ([B*S][3E], the three projections stacked)
-  if (!linear(s, x, w_qkv, b_qkv, qkv, rows, 3 * E, E, lt)) return CPATTN_ERR_CUDA;
+  if (!gemm(s, x, w_qkv, b_qkv, qkv, rows, 3 * E, E, 0, 0)) return CPATTN_ERR_CUDA;
   if (!heads(s, qkv, q, k, v, B, S, 3, H, D, 1)) return CPATTN_ERR_CUDA;
   st = cpattn_fwd(q, k, v, o, lse, B, H, S, D, cp_size, causal, scale, CPATTN_BF16, stream);
   if (st != CPATTN_OK) return st;
   if (!heads(s, om, o, nullptr, nullptr, B, S, 1, H, D, 0)) return CPATTN_ERR_CUDA;
-  if (!linear(s, om, w_o, b_o, y, rows, E, E, lt)) return CPATTN_ERR_CUDA;
+  if (!gemm(s, om, w_o, b_o, y, rows, E, E, 0, 0)) return CPATTN_ERR_CUDA;
   return CPATTN_OK;
 }
 
@@ -283,14 +224,14 @@ int cpattn_layer_bwd(const void* x, const void* w_qkv, const void* w_o, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void *dqkv = ws + w.qkv, *om = ws + w.om, *dom = ws + w.dom, *dout = ws + w.dout;
-  void *dq = ws + w.dq, *dk = ws + w.dk, *dv = ws + w.dv, *attn = ws + w.attn, *lt = ws + w.lt;
+  void *dq = ws + w.dq, *dk = ws + w.dk, *dv = ws + w.dv, *attn = ws + w.attn;
   float* part = reinterpret_cast<float*>(ws + w.part);
   const int rows = B * S;
   // output projection: dWo = dY^T Om, dbo = colsum(dY), dOm = dY Wo
   if (!heads(s, om, const_cast<void*>(o), nullptr, nullptr, B, S, 1, H, D, 0)) return CPATTN_ERR_CUDA;
-  if (!gemm(s, false, true, E, E, rows, om, E, dy, E, dw_o, E, nullptr, lt)) return CPATTN_ERR_CUDA;
+  if (!gemm(s, dy, om, nullptr, dw_o, E, E, rows, 1, 1)) return CPATTN_ERR_CUDA;
   if (!colsum(s, dy, db_o, rows, E, part)) return CPATTN_ERR_CUDA;
-  if (!gemm(s, false, false, E, rows, E, w_o, E, dy, E, dom, E, nullptr, lt)) return CPATTN_ERR_CUDA;
+  if (!gemm(s, dy, w_o, nullptr, dom, rows, E, E, 0, 1)) return CPATTN_ERR_CUDA;
   // attention backward on the per-head view of dOm
   if (!heads(s, dom, dout, nullptr, nullptr, B, S, 1, H, D, 1)) return CPATTN_ERR_CUDA;
   st = cpattn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, S, D, cp_size, causal, scale, attn,
@@ -299,10 +240,23 @@ int cpattn_layer_bwd(const void* x, const void* w_qkv, const void* w_o, const vo
   // input projection: dQKV = [dQ|dK|dV] per row, dWqkv = dQKV^T X,
   // dbqkv = colsum(dQKV), dX = dQKV Wqkv
   if (!heads(s, dqkv, dq, dk, dv, B, S, 3, H, D, 0)) return CPATTN_ERR_CUDA;
-  if (!gemm(s, false, true, E, 3 * E, rows, x, E, dqkv, 3 * E, dw_qkv, E, nullptr, lt)) return CPATTN_ERR_CUDA;
+  if (!gemm(s, dqkv, x, nullptr, dw_qkv, 3 * E, E, rows, 1, 1)) return CPATTN_ERR_CUDA;
   if (!colsum(s, dqkv, db_qkv, rows, 3 * E, part)) return CPATTN_ERR_CUDA;
-  if (!gemm(s, false, false, E, rows, 3 * E, w_qkv, E, dqkv, 3 * E, dx, E, nullptr, lt)) return CPATTN_ERR_CUDA;
+  if (!gemm(s, dqkv, w_qkv, nullptr, dx, rows, E, 3 * E, 0, 1)) return CPATTN_ERR_CUDA;
   return CPATTN_OK;
+}
+
+int cpattn_gemm(const void* A, const void* B, const void* bias, void* C, int M, int N, int K,
+                int a_layout, int b_layout, void* stream) {
+  NvtxRange nv("cpattn_gemm");
+  if (gemm_check(M, N, K) != 0) return CPATTN_ERR_SHAPE;
+  if ((a_layout != 0 && a_layout != 1) || (b_layout != 0 && b_layout != 1)) return CPATTN_ERR_ARG;
+  if (!A || !B || !C) return CPATTN_ERR_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C) || (bias && !aligned16(bias)))
+    return CPATTN_ERR_ALIGN;
+  return gemm(static_cast<cudaStream_t>(stream), A, B, bias, C, M, N, K, a_layout, b_layout)
+             ? CPATTN_OK
+             : CPATTN_ERR_CUDA;
 }
 
 }  // extern "C"
