@@ -359,6 +359,48 @@ def time_workload(cp, w, dev, peaks, steps=5, warmup=3):
     return out
 
 
+def time_fp8_fwd(cp, w, q, k, v, peaks, steps=10, warmup=3):
+    """The e4m3 ring forward (cpattn_fwd_fp8) on the workload's inputs, already
+    quantised (K/V kept in e4m3, as a context-parallel job would hold them),
+    and, separately, the quantisation of q, k, v (amax + codes, V transposed)."""
+    import torch
+    dev = q.device
+    stream = torch.cuda.current_stream(dev)
+    q8, k8, vt8, a3 = cp.quantize_qkv_e4m3(q, k, v)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps
+
+    n0 = cp.launch_count()
+    fwd_ms = timed(lambda: cp.fwd_fp8(q8, k8, vt8, a3, w.cp_size, w.causal, w.scale, out=o, lse=lse))
+    n_fwd = (cp.launch_count() - n0) / (steps + warmup)
+    quant_ms = timed(lambda: cp.quantize_qkv_e4m3(q, k, v))
+    st = cp.sync_status()
+    if st != cp.OK:
+        raise RuntimeError(f"fp8 forward failed: {cp.status_str(st)}")
+    tfl = w.flops_fwd() / (fwd_ms * 1e-3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    del q8, k8, vt8, a3, o, lse
+    return {"kernel": "tc_fwd_kernel<128, e4m3>", "workload": w.name, "ms": fwd_ms, "tflops": tfl,
+            "launches_per_call": n_fwd,
+            "roofline": {"bound": "tensor", "achieved": tfl, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": tfl / fp8_peak,
+                         "peak_kind": f"2 x bf16_tflops ({peaks['source']}; nominal fp8/bf16 dense ratio 4.5/2.25)"},
+            "quantize_ms": quant_ms,
+            "tflops_incl_quantize": w.flops_fwd() / ((fwd_ms + quant_ms) * 1e-3) / 1e12}
+
+
 # --------------------------------------------------------------- GPU arm --
 def run_gpu(args, w):
     import torch
@@ -530,8 +572,10 @@ def run_gpu(args, w):
 
     # ---- the other workloads and the standalone merge (device-timed, after the
     # headline region; each its own allocation) ----
-    per_config, merge = None, None
+    per_config, merge, fp8 = None, None, None
     if not args.no_extra and world == 1:
+        if w.D == 128 and w.dtype == "bf16":
+            fp8 = time_fp8_fwd(cp, w, qd, kd, vd, peaks)
         per_config = {}
         from long_sequence_context_b200.inputs import WORKLOADS
         for name, wk in WORKLOADS.items():
@@ -563,6 +607,7 @@ def run_gpu(args, w):
             "roofline": roof,
             "per_config": per_config,
             "merge": merge,
+            "fp8_fwd": fp8,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,

@@ -179,6 +179,41 @@ int cpattn_bwd_accumulate(const void* q, const void* k, const void* v, const voi
                           float scale, void* workspace, size_t ws_bytes, int dtype,
                           void* stream);
 
+/*
+ * FP8 (e4m3) forward.  "Megatron-LM source analysis: Context Parallel",
+ * section 4: FP8 attention inputs combined with context parallelism, to save
+ * memory.  The pages fix neither the format nor the scaling; this library
+ * uses e4m3 ("fn": largest finite 448, no infinities) with one scale per
+ * tensor:
+ *     s = 448 / max|x|  (fp32; 1 for an all-zero tensor),
+ *     code = e4m3(fp32(x * s)), round to nearest even, saturating to +-448,
+ * and the value a code stands for is code / s.  The attention computed is the
+ * attention of those values, with P = softmax rounded to e4m3 (scaled by 2^6)
+ * before the P.V product; O is bf16, LSE fp32 as in cpattn_fwd.
+ *
+ * cpattn_amax -- *amax (device fp32) = max_i |x[i]| over n elements of dtype.
+ *   amax must be 4-byte aligned; the call zeroes it first (cudaMemsetAsync on
+ *   `stream`), so it needs no initialisation.
+ * cpattn_quantize_e4m3 -- codes of x ([BH][S][D], dtype) with the scale
+ *   derived from *amax (device, as written by cpattn_amax):
+ *     transpose = 0: out [BH][S][D] bytes (the layout of q and k)
+ *     transpose = 1: out [BH][D][S] bytes (V transposed per head); S % 64 == 0
+ *   D in {64, 128}; x and out 16-byte aligned.
+ * cpattn_fwd_fp8 -- the ring forward of cpattn_fwd on e4m3 inputs:
+ *     q8, k8 : [B][H][S][D] codes;  vt8: [B][H][D][S] codes (V transposed)
+ *     amax   : device float[3] = max|q|, max|k|, max|v| (the scales' source)
+ *     o      : [B][H][S][D] bf16;   lse: [B][H][S] fp32 (written)
+ *   Preconditions: those of cpattn_fwd, and D == 128 and a chunk length that
+ *   is a multiple of 128 (CPATTN_ERR_SHAPE).  Pointers 16-byte aligned (amax:
+ *   4).  One tcgen05 launch (kind::f8f6f4 MMAs).
+ */
+int cpattn_amax(const void* x, long n, int dtype, float* amax, void* stream);
+int cpattn_quantize_e4m3(const void* x, int dtype, int BH, int S, int D, int transpose,
+                         const float* amax, uint8_t* out, void* stream);
+int cpattn_fwd_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* vt8, const float* amax,
+                   void* o, float* lse, int B, int H, int S, int D, int cp_size, int causal,
+                   float scale, void* stream);
+
 /* Size of the fixed device scratch array used by cpattn_bwd_noalloc (64 MiB). */
 #define CPATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
 
@@ -324,7 +359,8 @@ long long cpattn_launch_count(void);
  *   preprocess (delta), 5 CUDA-core dK/dV, 6 CUDA-core dQ, 7 tcgen05 dK/dV,
  *   8 tcgen05 dQ, 9 layer head split / merge, 10 layer bias gradients,
  *   11 gradient accumulation (cpattn_accumulate), 12 GEMM (cpattn_gemm and
- *   the layer's projections).
+ *   the layer's projections), 13 tcgen05 e4m3 forward (cpattn_fwd_fp8),
+ *   14 max|x| and e4m3 quantisation.
  */
 int cpattn_profile(int on);
 int cpattn_profile_read(int kernel_kind, double* total_ms, long long* launches);

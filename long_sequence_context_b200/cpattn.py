@@ -25,7 +25,8 @@ EXPORTS = ["cpattn_plan", "cpattn_fwd", "cpattn_fwd_step", "cpattn_merge", "cpat
            "cpattn_status_str", "cpattn_launch_count", "cpattn_set_path", "cpattn_last_path",
            "cpattn_debug_stall", "cpattn_profile", "cpattn_profile_read", "cpattn_bwd_noalloc",
            "cpattn_layer_workspace_bytes", "cpattn_layer_fwd", "cpattn_layer_bwd",
-           "cpattn_accumulate", "cpattn_bwd_accumulate", "cpattn_gemm"]
+           "cpattn_accumulate", "cpattn_bwd_accumulate", "cpattn_gemm", "cpattn_amax",
+           "cpattn_quantize_e4m3", "cpattn_fwd_fp8"]
 
 # size of the library's fixed scratch array behind bwd_noalloc
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -65,6 +66,9 @@ def _load():
         "cpattn_accumulate": ([vp, vp, l, i, vp], i),
         "cpattn_layer_fwd": ([vp] * 11 + [i] * 6 + [f, vp, sz, vp], i),
         "cpattn_gemm": ([vp, vp, vp, vp, i, i, i, i, i, vp], i),
+        "cpattn_amax": ([vp, l, i, vp, vp], i),
+        "cpattn_quantize_e4m3": ([vp, i, i, i, i, i, vp, vp, vp], i),
+        "cpattn_fwd_fp8": ([vp] * 6 + [i] * 6 + [f, vp], i),
         "cpattn_layer_bwd": ([vp] * 14 + [i] * 6 + [f, vp, sz, vp], i),
     }
     for name, (args, res) in sigs.items():
@@ -332,6 +336,75 @@ def gemm(a, b, bias=None, a_t: bool = False, b_t: bool = False, out=None, stream
     return c
 
 
+def amax(x, out=None, stream=None):
+    """max |x| as a one-element fp32 device tensor (or into `out`)."""
+    if not isinstance(x, torch.Tensor):
+        raise TypeError("x must be a torch.Tensor")
+    _dtype_code(x)
+    _expect(x, "x", x.shape, x.dtype)
+    if out is not None:
+        _expect(out, "out", (1,), torch.float32, x)
+    a = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib.cpattn_amax(_dev(x, "x"), x.numel(), _dtype_code(x), _dev(a, "amax"), _stream(stream)),
+           "cpattn_amax")
+    return a
+
+
+def quantize_e4m3(x, amax_t, transpose: bool = False, stream=None):
+    """e4m3 codes (uint8) of x [B, H, S, D] with s = 448 / amax_t (device fp32
+    scalar, e.g. from amax()): [B, H, S, D], or [B, H, D, S] with transpose."""
+    if not isinstance(x, torch.Tensor) or x.dim() != 4:
+        raise ValueError("x must be a [B, H, S, D] tensor")
+    _dtype_code(x)
+    _expect(x, "x", x.shape, x.dtype)
+    if not isinstance(amax_t, torch.Tensor) or amax_t.numel() < 1 or amax_t.dtype != torch.float32 \
+            or amax_t.device != x.device:
+        raise ValueError("amax_t must be a float32 tensor on x's device")
+    B, H, S, D = x.shape
+    shape = (B, H, D, S) if transpose else (B, H, S, D)
+    out = torch.empty(shape, dtype=torch.uint8, device=x.device)
+    _check(lib.cpattn_quantize_e4m3(_dev(x, "x"), _dtype_code(x), B * H, S, D, int(transpose),
+                                    ctypes.c_void_p(amax_t.data_ptr()), _dev(out, "out"),
+                                    _stream(stream)), "cpattn_quantize_e4m3")
+    return out
+
+
+def quantize_qkv_e4m3(q, k, v, stream=None):
+    """(q8, k8, vt8, amax3): per-tensor e4m3 codes of q, k and of V transposed
+    per head, and the device float[3] of max|q|, max|k|, max|v|."""
+    B, H, S, D = _qkv(q, k, v)
+    a3 = torch.empty(3, dtype=torch.float32, device=q.device)
+    for i, t in enumerate((q, k, v)):
+        amax(t, out=a3[i:i + 1], stream=stream)
+    q8 = quantize_e4m3(q, a3[0:1], stream=stream)
+    k8 = quantize_e4m3(k, a3[1:2], stream=stream)
+    vt8 = quantize_e4m3(v, a3[2:3], transpose=True, stream=stream)
+    return q8, k8, vt8, a3
+
+
+def fwd_fp8(q8, k8, vt8, amax3, cp_size: int, causal: bool = True, scale=None, out=None, lse=None,
+            stream=None):
+    """Ring forward on e4m3 inputs (see quantize_qkv_e4m3): returns (o bf16, lse fp32)."""
+    if not isinstance(q8, torch.Tensor) or q8.dim() != 4:
+        raise ValueError("q8 must be a [B, H, S, D] tensor")
+    B, H, S, D = q8.shape
+    _expect(q8, "q8", (B, H, S, D), torch.uint8)
+    _expect(k8, "k8", (B, H, S, D), torch.uint8, q8)
+    _expect(vt8, "vt8", (B, H, D, S), torch.uint8, q8)
+    _expect(amax3, "amax3", (3,), torch.float32, q8)
+    scale = float(scale if scale is not None else D ** -0.5)
+    if out is not None:
+        _expect(out, "out", (B, H, S, D), torch.bfloat16, q8)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, S), torch.float32, q8)
+    o = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=q8.device) if out is None else out
+    l_t = torch.empty((B, H, S), dtype=torch.float32, device=q8.device) if lse is None else lse
+    _check(lib.cpattn_fwd_fp8(_dev(q8, "q8"), _dev(k8, "k8"), _dev(vt8, "vt8"), _dev(amax3, "amax3"),
+                              _dev(o, "o"), _dev(l_t, "lse"), B, H, S, D, cp_size, int(causal), scale,
+                              _stream(stream)), "cpattn_fwd_fp8")
+    return o, l_t
+
+
 def layer_workspace_bytes(B, S, E, H) -> int:
     return int(lib.cpattn_layer_workspace_bytes(B, S, E, H))
 
@@ -422,7 +495,8 @@ def debug_stall(n: int) -> int:
 
 KERNEL_KINDS = {0: "tc_fwd", 1: "simt_fwd", 2: "merge", 3: "finalize", 4: "bwd_delta",
                 5: "simt_dkdv", 6: "simt_dq", 7: "tc_dkdv", 8: "tc_dq", 9: "layer_heads",
-                10: "layer_colsum", 11: "accumulate", 12: "gemm"}
+                10: "layer_colsum", 11: "accumulate", 12: "gemm", 13: "tc_fwd_fp8",
+                14: "quant_e4m3"}
 
 
 def profile(on: bool) -> int:

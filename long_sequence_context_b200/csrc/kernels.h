@@ -51,6 +51,10 @@ int launch_tc_bwd(const AttnShape& sh, const void* q, const void* k, const void*
                   const void* o, const float* lse, const void* dout, void* dq, void* dk,
                   void* dv, float* ws_delta, float* ws_lse2, int acc_f32, unsigned* err,
                   cudaStream_t stream);
+// e4m3 forward (D = 128): q8, k8 [B*H*S][D] codes, vt8 [B*H*D][S] codes (V
+// transposed per head), amax: device max|q|, max|k|, max|v|; o bf16.
+int launch_tc_fwd_fp8(const AttnShape& sh, const void* q8, const void* k8, const void* vt8,
+                      const float* amax, void* o, float* lse, unsigned* err, cudaStream_t stream);
 bool tc_fwd_supported(const AttnShape& sh);
 bool tc_bwd_supported(const AttnShape& sh);
 
@@ -106,7 +110,9 @@ enum KernelId : int {
   kKLayerColsum = 10, // bias gradients of the attention layer
   kKAccumulate = 11,  // fp32 gradient sums of the multi-rank ring backward
   kKGemm = 12,        // projection GEMMs of the attention layer (cpattn_gemm)
-  kKNumKernels = 13
+  kKTcFwdFp8 = 13,    // tcgen05 forward on e4m3 inputs (cpattn_fwd_fp8)
+  kKQuant = 14,       // max|x| and e4m3 quantisation (cpattn_amax, cpattn_quantize_e4m3)
+  kKNumKernels = 15
 };
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);

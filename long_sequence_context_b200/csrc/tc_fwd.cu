@@ -22,6 +22,16 @@
 // the P.V MMA straight from TMEM.
 // Per K/V tile j the MMA thread issues PV0(j-1), S0(j), PV1(j-1), S1(j), so
 // softmax of one Q tile overlaps the MMAs of the other.
+//
+// FP8 variant (F8 = true, D = 128; "Megatron-LM source analysis: Context
+// Parallel", section 4: FP8 attention inputs under context parallelism): Q, K
+// and V^T arrive as e4m3 codes with per-tensor scales (code = e4m3(x * s),
+// s = 448 / max|x|), the two products run as kind::f8f6f4 MMAs (K = 32 per
+// instruction), V is stored transposed per head ([d][key]) so that both
+// operands of P.V are K-major, and P is written back to TMEM as e4m3 (four per
+// column) scaled by 2^6.  The running maximum is then kept within 2^2 of the
+// true one, so the scaled P stays <= 2^8 < 448; the row sum l is taken from
+// the unrounded P.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,21 +51,26 @@ using namespace sm100;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // keep a stale row maximum unless the new one exceeds it by more than 2^8
+// (bf16 P) or 2^2 (e4m3 P, which must stay below 448 after its 2^6 scale)
 constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThresholdF8 = 2.0f;
+constexpr float kP8Log2Scale = 6.0f;  // e4m3 P holds 2^6 * P
 
-template <int D>
+template <int D, bool F8>
 struct FwdCfg {
   static constexpr int kTile = 128;                       // rows per Q / K / V tile
-  static constexpr int kTileBytes = kTile * D * 2;        // bf16 tile
-  static constexpr int kSubBytes = kTile * 128;           // one 64-column swizzled block
-  static constexpr int kStages = D == 128 ? 5 : 8;        // K/V slots
+  static constexpr int kElem = F8 ? 1 : 2;                // bytes per element
+  static constexpr int kTileBytes = kTile * D * kElem;    // one Q / K / V tile
+  static constexpr int kSubBytes = kTile * 128;           // one 128-byte-wide swizzled block
+  static constexpr int kStages = F8 ? 10 : (D == 128 ? 5 : 8);  // K/V slots
   static constexpr int kThreads = 384;
   static constexpr int kRegsSoftmax = 208;  // 2*128*208 + 128*80 <= 384*168
   static constexpr int kRegsOther = 80;
   static constexpr int kBarOffset = 2 * kTileBytes + kStages * kTileBytes;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
-  static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
-  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+  static constexpr uint32_t kIdescQK = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
+  static constexpr uint32_t kIdescPV = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
+  static_assert(!F8 || D == 128, "the e4m3 path takes D = 128 (one 128-byte swizzled row)");
 };
 
 struct FwdParams {
@@ -70,6 +85,7 @@ struct FwdParams {
   float sl2;       // scale * log2(e)
   void* o;
   float* lse;
+  const float* amax;  // e4m3 path: device max|q|, max|k|, max|v| (the scales' source)
   unsigned* err;
   int stall;       // omit one K load in CTA 0 (failure-detection tests)
 };
@@ -154,11 +170,17 @@ __device__ __forceinline__ int snake_item(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
-template <int D>
+// Per-tensor e4m3 scale 448 / amax (1 for an all-zero tensor), as the
+// quantiser computes it.
+__device__ __forceinline__ float e4m3_scale(float amax) {
+  return amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+}
+
+template <int D, bool F8>
 __global__ void __launch_bounds__(384, 1)
     tc_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams P) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -213,6 +235,15 @@ __global__ void __launch_bounds__(384, 1)
   if (warp < 8) {
     // ------------------------------------------------------------ softmax --
     regs_inc<C::kRegsSoftmax>();
+    // scores arrive as products of codes: undo the q and k scales; the output
+    // undoes the v scale
+    float sl2 = P.sl2, out_mul = 1.f;
+    if constexpr (F8) {
+      sl2 = P.sl2 / (e4m3_scale(P.amax[0]) * e4m3_scale(P.amax[1]));
+      out_mul = 1.f / e4m3_scale(P.amax[2]);
+    }
+    constexpr float kThresh = F8 ? kRescaleThresholdF8 : kRescaleThreshold;
+    constexpr float kPOff = F8 ? kP8Log2Scale : 0.f;
     const int wg = warp >> 2;               // which Q tile
     const int quarter = warp & 3;           // TMEM lane quarter of this warp
     const int rloc = quarter * 32 + lane;   // row within the 128-row tile
@@ -259,9 +290,9 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 8; ++i) mp[i] = fmaxf(mp[i], __uint_as_float(r[c + i]));
         const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                                fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-        const float m_tile = mx * P.sl2;
+        const float m_tile = mx * sl2;
         float m_new = m;
-        if (m_tile > m + kRescaleThreshold || m == -INFINITY) m_new = fmaxf(m, m_tile);
+        if (m_tile > m + kThresh || m == -INFINITY) m_new = fmaxf(m, m_tile);
         const bool grow = (m != -INFINITY) && (m_new > m);
         const float f = grow ? ex2(m - m_new) : 1.f;
         l *= f;
@@ -269,18 +300,30 @@ __global__ void __launch_bounds__(384, 1)
         // (factor 1 for rows whose maximum stayed) when any row needs it
         if (j > 0 && __any_sync(0xffffffffu, grow)) rescale_rows<D>(tO, f);
         m = m_new;
-        const float base = (m == -INFINITY) ? 0.f : m;
+        const float base = ((m == -INFINITY) ? 0.f : m) - kPOff;
         float ls[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
+        if constexpr (F8) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = ex2(fmaf(__uint_as_float(r[c]), P.sl2, -base));
-          const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), P.sl2, -base));
-          ls[(c >> 1) & 3] += p0 + p1;
-          r[c >> 1] = pack_bf16x2(p0, p1);  // r[c/2] was read at or before this step
+          for (int c = 0; c < 128; c += 4) {
+            const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, -base));
+            const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, -base));
+            const float p2 = ex2(fmaf(__uint_as_float(r[c + 2]), sl2, -base));
+            const float p3 = ex2(fmaf(__uint_as_float(r[c + 3]), sl2, -base));
+            ls[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
+            r[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);  // r[c/4] was read at or before this step
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, -base));
+            const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, -base));
+            ls[(c >> 1) & 3] += p0 + p1;
+            r[c >> 1] = pack_bf16x2(p0, p1);  // r[c/2] was read at or before this step
+          }
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tmem_st32<0>(tS + 0, r);
-        tmem_st32<32>(tS + 32, r);
+        if constexpr (!F8) tmem_st32<32>(tS + 32, r);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_ready[wg]);
@@ -308,7 +351,7 @@ __global__ void __launch_bounds__(384, 1)
       if (!mbar_wait_warp(&o_ready[wg], o_cnt & 1, abort_flag, P.err)) break;
       ++o_cnt;
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = out_mul / l;
 #pragma unroll
       for (int cb = 0; cb < D; cb += 32) {
         uint32_t ov[32];
@@ -335,7 +378,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (store) P.lse[orow] = (m + __log2f(l)) * kLn2;
+      if (store) P.lse[orow] = (m + __log2f(l) - kPOff) * kLn2;
       tc_fence_before();
     }
   } else {
@@ -360,10 +403,15 @@ __global__ void __launch_bounds__(384, 1)
       const int rowbase = it.bh * S;
       if (lane == 0) {
         mbar_expect_tx(q_full, 2 * C::kTileBytes);
+        if constexpr (F8) {
+          tma_load_2d(sQ[0], &tmQ, q_full, 0, rowbase + it.qt0 * 128);
+          tma_load_2d(sQ[1], &tmQ, q_full, 0, rowbase + it.qt1 * 128);
+        } else {
 #pragma unroll
-        for (int sb = 0; sb < D / 64; ++sb) {
-          tma_load_2d(sQ[0] + sb * C::kSubBytes, &tmQ, q_full, sb * 64, rowbase + it.qt0 * 128);
-          tma_load_2d(sQ[1] + sb * C::kSubBytes, &tmQ, q_full, sb * 64, rowbase + it.qt1 * 128);
+          for (int sb = 0; sb < D / 64; ++sb) {
+            tma_load_2d(sQ[0] + sb * C::kSubBytes, &tmQ, q_full, sb * 64, rowbase + it.qt0 * 128);
+            tma_load_2d(sQ[1] + sb * C::kSubBytes, &tmQ, q_full, sb * 64, rowbase + it.qt1 * 128);
+          }
         }
       }
       ++n_items;
@@ -380,11 +428,19 @@ __global__ void __launch_bounds__(384, 1)
               stall = false;  // this K tile is never loaded: the consumer's wait runs out
             } else {
               mbar_expect_tx(&kv_full[s], C::kTileBytes);
-              const CUtensorMap* map = which ? &tmV : &tmK;
+              if constexpr (F8) {
+                // K: [key rows][d] codes; V^T: [d rows][key] codes of this head
+                if (which)
+                  tma_load_2d(sKV + s * C::kTileBytes, &tmV, &kv_full[s], tile * 128, it.bh * D);
+                else
+                  tma_load_2d(sKV + s * C::kTileBytes, &tmK, &kv_full[s], 0, rowbase + tile * 128);
+              } else {
+                const CUtensorMap* map = which ? &tmV : &tmK;
 #pragma unroll
-              for (int sb = 0; sb < D / 64; ++sb)
-                tma_load_2d(sKV + s * C::kTileBytes + sb * C::kSubBytes, map, &kv_full[s], sb * 64,
-                            rowbase + tile * 128);
+                for (int sb = 0; sb < D / 64; ++sb)
+                  tma_load_2d(sKV + s * C::kTileBytes + sb * C::kSubBytes, map, &kv_full[s],
+                              sb * 64, rowbase + tile * 128);
+              }
             }
           }
           __syncwarp();
@@ -411,20 +467,35 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t aKV = smem_u32(sKV);
     // one descriptor per operand tile; k-steps are constant offsets from it
     const uint64_t dQd[2] = {smem_desc_sw128(aQ[0], 16, 1024), smem_desc_sw128(aQ[1], 16, 1024)};
-    // O += P V: A = P (bf16, two per TMEM column), B = V (MN-major over d)
+    // O += P V: A = P (bf16, two per TMEM column), B = V (MN-major over d);
+    // e4m3: A = P (four per TMEM column), B = V^T (K-major over keys)
     auto issue_pv = [&](uint32_t t_o, uint32_t t_p, uint32_t slot_v, bool first) {
-      const uint64_t dv = smem_desc_sw128(aKV + slot_v * C::kTileBytes, C::kSubBytes, 1024);
+      if constexpr (F8) {
+        const uint64_t dv = smem_desc_sw128(aKV + slot_v * C::kTileBytes, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts(t_o, t_p + kk * 8, desc_at(dv, kk * 2048), C::kIdescPV, (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts_f8(t_o, t_p + kk * 8, desc_at(dv, kk * 32), C::kIdescPV,
+                    (first && kk == 0) ? 0u : 1u);
+      } else {
+        const uint64_t dv = smem_desc_sw128(aKV + slot_v * C::kTileBytes, C::kSubBytes, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(t_o, t_p + kk * 8, desc_at(dv, kk * 2048), C::kIdescPV, (first && kk == 0) ? 0u : 1u);
+      }
     };
-    // S = Q K^T: both operands K-major
+    // S = Q K^T: both operands K-major (bf16: 16 per k-step, e4m3: 32)
     auto issue_qk = [&](uint32_t t_s, uint64_t dq, uint32_t slot_k) {
       const uint64_t dk = smem_desc_sw128(aKV + slot_k * C::kTileBytes, 16, 1024);
+      if constexpr (F8) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-        mma_ss(t_s, desc_at(dq, off), desc_at(dk, off), C::kIdescQK, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss_f8(t_s, desc_at(dq, kk * 32), desc_at(dk, kk * 32), C::kIdescQK, kk > 0 ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+          mma_ss(t_s, desc_at(dq, off), desc_at(dk, off), C::kIdescQK, kk > 0 ? 1u : 0u);
+        }
       }
     };
     uint32_t kv_idx = 0, p_cnt = 0, n_items = 0;
@@ -518,16 +589,23 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D>
+template <int D, bool F8>
 int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v, void* o,
-                float* lse, unsigned* err, int stall, int t0, int t1, int out_f32,
-                cudaStream_t stream) {
-  using C = FwdCfg<D>;
+                float* lse, const float* amax, unsigned* err, int stall, int t0, int t1,
+                int out_f32, cudaStream_t stream) {
+  using C = FwdCfg<D, F8>;
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)sh.B * sh.H * sh.S;
-  if (!make_tmap_bf16_2d(&mq, q, rows, D, 64, 128) || !make_tmap_bf16_2d(&mk, k, rows, D, 64, 128) ||
-      !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128))
-    return -1;
+  if constexpr (F8) {
+    // q, k: [B*H*S][D] codes; v: V^T, [B*H*D][S] codes
+    if (!make_tmap_u8_2d(&mq, q, rows, D, 128, 128) || !make_tmap_u8_2d(&mk, k, rows, D, 128, 128) ||
+        !make_tmap_u8_2d(&mv, v, (uint64_t)sh.B * sh.H * D, sh.S, 128, 128))
+      return -1;
+  } else {
+    if (!make_tmap_bf16_2d(&mq, q, rows, D, 64, 128) || !make_tmap_bf16_2d(&mk, k, rows, D, 64, 128) ||
+        !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128))
+      return -1;
+  }
   FwdParams P;
   P.g = sh.g;
   P.BH = sh.B * sh.H;
@@ -541,17 +619,19 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.sl2 = sh.scale * kLog2e;
   P.o = o;
   P.lse = lse;
+  P.amax = amax;
   P.err = err;
   P.stall = stall;
   static std::atomic<unsigned long long> attr_done{0};
-  if (!smem_attr_once(tc_fwd_kernel<D>, C::kSmemBytes, attr_done)) return -1;
+  if (!smem_attr_once(tc_fwd_kernel<D, F8>, C::kSmemBytes, attr_done)) return -1;
   int dev = 0;
   cudaGetDevice(&dev);
   int grid = num_sms(dev);
   if (grid > P.n_items) grid = P.n_items;
-  prof_begin(kKTcFwd, stream);
-  tc_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, P);
-  prof_end(kKTcFwd, stream);
+  const int prof_id = F8 ? kKTcFwdFp8 : kKTcFwd;
+  prof_begin(prof_id, stream);
+  tc_fwd_kernel<D, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, P);
+  prof_end(prof_id, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
 
@@ -567,16 +647,25 @@ bool tc_fwd_supported(const AttnShape& sh) {
 
 int launch_tc_fwd(const AttnShape& sh, const void* q, const void* k, const void* v, void* o,
                   float* lse, unsigned* err, int stall, cudaStream_t stream) {
-  if (sh.D == 64) return launch_impl<64>(sh, q, k, v, o, lse, err, stall, 0, sh.g.N, 0, stream);
-  return launch_impl<128>(sh, q, k, v, o, lse, err, stall, 0, sh.g.N, 0, stream);
+  if (sh.D == 64)
+    return launch_impl<64, false>(sh, q, k, v, o, lse, nullptr, err, stall, 0, sh.g.N, 0, stream);
+  return launch_impl<128, false>(sh, q, k, v, o, lse, nullptr, err, stall, 0, sh.g.N, 0, stream);
 }
 
 int launch_tc_fwd_step(const AttnShape& sh, const void* q, const void* k, const void* v,
                        float* o_part, float* lse_part, int step, unsigned* err,
                        cudaStream_t stream) {
   if (sh.D == 64)
-    return launch_impl<64>(sh, q, k, v, o_part, lse_part, err, 0, step, step + 1, 1, stream);
-  return launch_impl<128>(sh, q, k, v, o_part, lse_part, err, 0, step, step + 1, 1, stream);
+    return launch_impl<64, false>(sh, q, k, v, o_part, lse_part, nullptr, err, 0, step, step + 1, 1,
+                                  stream);
+  return launch_impl<128, false>(sh, q, k, v, o_part, lse_part, nullptr, err, 0, step, step + 1, 1,
+                                 stream);
+}
+
+int launch_tc_fwd_fp8(const AttnShape& sh, const void* q8, const void* k8, const void* vt8,
+                      const float* amax, void* o, float* lse, unsigned* err, cudaStream_t stream) {
+  if (sh.D != 128) return -1;
+  return launch_impl<128, true>(sh, q8, k8, vt8, o, lse, amax, err, 0, 0, sh.g.N, 0, stream);
 }
 
 }  // namespace cpattn

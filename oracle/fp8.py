@@ -74,11 +74,14 @@ def scale_of(amax) -> np.float32:
     return np.float32(E4M3_MAX) / amax
 
 
-def quantize(x):
+def quantize(x, amax=None):
     """(codes, s, amax) for a tensor x of bf16- or fp32-representable values:
-    amax = max|x|, s = 448 / amax (fp32), codes = encode(fp32(x * s))."""
+    amax = max|x| (or the given maximum of the whole tensor x is a part of),
+    s = 448 / amax (fp32), codes = encode(fp32(x * s))."""
     x32 = np.asarray(x, dtype=np.float32)
-    amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
+    if amax is None:
+        amax = np.max(np.abs(x32)) if x32.size else 0.0
+    amax = np.float32(amax)
     s = scale_of(amax)
     codes = encode((x32 * s).astype(np.float32))
     return codes, s, amax
