@@ -35,9 +35,9 @@
  *     are recorded on the device and reported by cpattn_sync_status().
  *   - Preconditions (CPATTN_ERR_SHAPE otherwise): B, H >= 1; S >= 1;
  *     cp_size >= 1; D is 64 or 128; causal: S % (2*cp_size) == 0, non-causal:
- *     S % cp_size == 0, and the chunk length c is a multiple of 16.  bf16
- *     problems with c % 128 == 0 run on the tcgen05 tensor-core kernels, the
- *     rest on the CUDA-core kernels.
+ *     S % cp_size == 0 (any chunk length c).  bf16 problems with c % 128 == 0
+ *     run on the tcgen05 tensor-core kernels, the rest (every fp32 problem,
+ *     bf16 chunks of other lengths) on the CUDA-core kernels.
  *   - Pointers must be 16-byte aligned (CPATTN_ERR_ALIGN); scale must be
  *     finite and > 0 (CPATTN_ERR_ARG).
  *   - Sizes are not visible through plain pointers: every buffer must hold the

@@ -73,7 +73,6 @@ int check_shape(int B, int H, int S, int D, int cp_size, int causal, float scale
   if (D != 64 && D != 128) return CPATTN_ERR_SHAPE;
   const int n_chunks = causal ? 2 * cp_size : cp_size;
   if (S % n_chunks != 0) return CPATTN_ERR_SHAPE;
-  if ((S / n_chunks) % 16 != 0) return CPATTN_ERR_SHAPE;
   if ((long long)B * H * S * D > (1LL << 40)) return CPATTN_ERR_SHAPE;
   if ((long long)B * H > 65535LL) return CPATTN_ERR_SHAPE;  // grid.y of the CUDA-core kernels
   sh->B = B;

@@ -74,7 +74,9 @@ __device__ __forceinline__ void out_f(T* p, float* acc, long i, float x) {
 constexpr int kTile = 16;   // keys (dK/dV kernel) or rows (dQ kernel) per block
 constexpr int kBatch = 8;   // rows / keys staged in shared memory at a time
 
-// grid (S/16, B*H), block 128: thread = (key t/8, d-slice t%8)
+// grid (n_chunks * ceil(c/16), B*H), block 128: thread = (key t/8, d-slice t%8).
+// Block x owns keys [j0, j0 + 16) of kv chunk x / ceil(c/16); keys at or past
+// the chunk's end read no input and write nothing.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                    const T* __restrict__ v,
@@ -89,19 +91,21 @@ __global__ void __launch_bounds__(128) dkdv_kernel(const T* __restrict__ q, cons
   __shared__ float Qs[kBatch][D], dOs[kBatch][D], Ls[kBatch], Ds[kBatch];
   const long bh = blockIdx.y;
   const long base = bh * (long)g.S * D;
-  const int j0 = blockIdx.x * kTile;
+  const int bpc = (g.c + kTile - 1) / kTile;
+  const int b = blockIdx.x / bpc;         // kv chunk of these keys
+  const int j0 = b * g.c + (blockIdx.x % bpc) * kTile;
   const int kj = threadIdx.x / 8, sl = threadIdx.x % 8;
   const int key = j0 + kj;
+  const bool key_in = key < (b + 1) * g.c;
   float kr[SL], vr[SL], dk_acc[SL], dv_acc[SL];
 #pragma unroll
   for (int i = 0; i < SL; ++i) {
-    kr[i] = ld_f(k, base + (long)key * D + sl * SL + i);
-    vr[i] = ld_f(v, base + (long)key * D + sl * SL + i);
+    kr[i] = key_in ? ld_f(k, base + (long)key * D + sl * SL + i) : 0.f;
+    vr[i] = key_in ? ld_f(v, base + (long)key * D + sl * SL + i) : 0.f;
     dk_acc[i] = 0.f;
     dv_acc[i] = 0.f;
   }
   const float scale_log2 = scale * kLog2e;
-  const int b = j0 / g.c;                 // kv chunk of these keys
   const int owner = chunk_owner(g, b);    // rank whose K/V these are
   for (int t = 0; t < g.N; ++t) {
     const int r = (owner + t) % g.N;      // rank holding this K/V at step t
@@ -148,6 +152,7 @@ __global__ void __launch_bounds__(128) dkdv_kernel(const T* __restrict__ q, cons
       }
     }
   }
+  if (!key_in) return;
 #pragma unroll
   for (int i = 0; i < SL; ++i) {
     out_f(dk, dk_acc_out, base + (long)key * D + sl * SL + i, dk_acc[i] * scale);
@@ -155,7 +160,9 @@ __global__ void __launch_bounds__(128) dkdv_kernel(const T* __restrict__ q, cons
   }
 }
 
-// grid (S/16, B*H), block 128: thread = (row t/8, d-slice t%8)
+// grid (n_chunks * ceil(c/16), B*H), block 128: thread = (row t/8, d-slice t%8).
+// Block x owns rows [i0, i0 + 16) of q chunk x / ceil(c/16); rows at or past
+// the chunk's end read no input and write nothing.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) dq_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                  const T* __restrict__ v,
@@ -168,20 +175,22 @@ __global__ void __launch_bounds__(128) dq_kernel(const T* __restrict__ q, const 
   __shared__ float Ks[kBatch][D], Vs[kBatch][D];
   const long bh = blockIdx.y;
   const long base = bh * (long)g.S * D;
-  const int i0 = blockIdx.x * kTile;
+  const int bpc = (g.c + kTile - 1) / kTile;
+  const int a = blockIdx.x / bpc;  // q chunk of these rows
+  const int i0 = a * g.c + (blockIdx.x % bpc) * kTile;
   const int ri = threadIdx.x / 8, sl = threadIdx.x % 8;
   const int row = i0 + ri;
+  const bool row_in = row < (a + 1) * g.c;
   float qr[SL], dor[SL], acc[SL];
 #pragma unroll
   for (int i = 0; i < SL; ++i) {
-    qr[i] = ld_f(q, base + (long)row * D + sl * SL + i);
-    dor[i] = ld_f(dout, base + (long)row * D + sl * SL + i);
+    qr[i] = row_in ? ld_f(q, base + (long)row * D + sl * SL + i) : 0.f;
+    dor[i] = row_in ? ld_f(dout, base + (long)row * D + sl * SL + i) : 0.f;
     acc[i] = 0.f;
   }
-  const float lse2 = lse[bh * g.S + row] * kLog2e;
-  const float dlt = delta[bh * g.S + row];
+  const float lse2 = row_in ? lse[bh * g.S + row] * kLog2e : INFINITY;
+  const float dlt = row_in ? delta[bh * g.S + row] : 0.f;
   const float scale_log2 = scale * kLog2e;
-  const int a = i0 / g.c;
   const int rank = chunk_owner(g, a);
   for (int t = 0; t < g.N; ++t) {
     const int src = step_src(g, rank, t);
@@ -220,6 +229,7 @@ __global__ void __launch_bounds__(128) dq_kernel(const T* __restrict__ q, const 
       }
     }
   }
+  if (!row_in) return;
 #pragma unroll
   for (int i = 0; i < SL; ++i) out_f(dq, dq_acc_out, base + (long)row * D + sl * SL + i, acc[i] * scale);
 }
@@ -238,7 +248,7 @@ int run_bwd(const AttnShape& sh, const void* q, const void* k, const void* v, co
   delta_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(O, dO, ws_delta, rows);
   prof_end(kKDelta, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
-  dim3 grid(sh.S / kTile, sh.B * sh.H);
+  dim3 grid(sh.g.n_chunks * ((sh.g.c + kTile - 1) / kTile), sh.B * sh.H);
   prof_begin(kKSimtDkdv, stream);
   float* acc_dk = acc_f32 ? static_cast<float*>(dk) : nullptr;
   float* acc_dv = acc_f32 ? static_cast<float*>(dv) : nullptr;

@@ -38,12 +38,15 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-constexpr int kRowsPerBlock = 16;  // 4 warps x 4 rows, all in one chunk
+constexpr int kRowsPerBlock = 16;  // 4 warps x 4 rows, all in one chunk (rows past its end idle)
 constexpr int kRowsPerWarp = 4;
 constexpr int kKeyTile = 32;       // one key per lane
 
-// grid: (S / 16, B*H), block 128.  Steps [t0, t1) of the ring for the 16 rows
-// of this block; online softmax in the log2 domain across every non-SKIP block.
+// grid: (n_chunks * ceil(c / 16), B*H), block 128.  Block x covers rows
+// [row0, row0 + 16) of chunk x / ceil(c / 16); rows at or past the chunk's end
+// read no input and write nothing, so any chunk length c works.  Steps
+// [t0, t1) of the ring; online softmax in the log2 domain across every
+// non-SKIP block.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) simt_fwd_kernel(const T* __restrict__ q,
                                                        const T* __restrict__ k,
@@ -58,11 +61,14 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const T* __restrict__ q,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long bh = blockIdx.y;
-  const int row0 = blockIdx.x * kRowsPerBlock;
+  const int bpc = (g.c + kRowsPerBlock - 1) / kRowsPerBlock;  // blocks per chunk
+  const int a = blockIdx.x / bpc;       // q chunk of this block
+  const int row0 = a * g.c + (blockIdx.x % bpc) * kRowsPerBlock;
+  const int row_end = (a + 1) * g.c;    // rows at or past it belong to the next chunk
   const long base = bh * (long)g.S * D;
 
   for (int idx = threadIdx.x; idx < kRowsPerBlock * D; idx += blockDim.x)
-    Qs[idx / D][idx % D] = to_f(q[base + (long)row0 * D + idx]);
+    Qs[idx / D][idx % D] = (row0 + idx / D < row_end) ? to_f(q[base + (long)row0 * D + idx]) : 0.f;
 
   float m[kRowsPerWarp], l[kRowsPerWarp], acc[kRowsPerWarp][DW];
 #pragma unroll
@@ -73,7 +79,6 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const T* __restrict__ q,
     for (int i = 0; i < DW; ++i) acc[r][i] = 0.f;
   }
 
-  const int a = row0 / g.c;             // q chunk of this block
   const int rank = chunk_owner(g, a);   // virtual rank holding it
   for (int t = t0; t < t1; ++t) {
     const int src = step_src(g, rank, t);
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(128) simt_fwd_kernel(const T* __restrict__ q,
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
     const int row = row0 + warp * kRowsPerWarp + r;
+    if (row >= row_end) continue;  // warp-uniform: the four rows of a warp are consecutive
     const long ro = base + (long)row * D;
     const bool empty = (l[r] == 0.f);
     const float inv = empty ? 0.f : 1.f / l[r];
@@ -214,7 +220,8 @@ int launch_simt_fwd(const AttnShape& sh, const void* q, const void* k, const voi
                     float* lse, int t0, int t1, int final_out, unsigned* err,
                     cudaStream_t stream) {
   (void)err;
-  dim3 grid(sh.S / kRowsPerBlock, sh.B * sh.H);
+  const int bpc = (sh.g.c + kRowsPerBlock - 1) / kRowsPerBlock;
+  dim3 grid(sh.g.n_chunks * bpc, sh.B * sh.H);
   const float sl2 = sh.scale * kLog2e;
   prof_begin(kKSimtFwd, stream);
   if (sh.bf16) {

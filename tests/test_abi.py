@@ -73,8 +73,8 @@ def _fwd_status(cp, S=256, D=128, cp_size=2, causal=1, scale=0.1, dtype=0, ptr=2
 
 
 def test_argument_errors_are_reported_before_launch(cp):
-    assert _fwd_status(cp, S=100) == cp.ERR_SHAPE          # not a multiple of 2*cp_size
-    assert _fwd_status(cp, S=2 * 2 * 8) == cp.ERR_SHAPE    # chunk of 8 rows
+    assert _fwd_status(cp, S=102) == cp.ERR_SHAPE          # not a multiple of 2*cp_size
+    assert _fwd_status(cp, S=2 * 2 * 8 + 2) == cp.ERR_SHAPE  # 34 rows: not 4 whole chunks
     assert _fwd_status(cp, D=96) == cp.ERR_SHAPE
     assert _fwd_status(cp, cp_size=0) == cp.ERR_SHAPE
     assert _fwd_status(cp, B=0) == cp.ERR_SHAPE
@@ -117,7 +117,7 @@ def test_layer_argument_errors_are_reported_before_launch(cp):
     assert fwd(scale=0.0) == cp.ERR_ARG
     assert fwd(ws=None) == cp.ERR_WORKSPACE
     assert fwd(ws_bytes=need - 1) == cp.ERR_WORKSPACE
-    assert fwd(S=100, ws_bytes=cp.layer_workspace_bytes(B, 100, E, H)) == cp.ERR_SHAPE  # chunk of 25 rows
+    assert fwd(S=100, ws_bytes=cp.layer_workspace_bytes(B, 100, E, H)) == cp.ERR_SHAPE  # B*S % 8 != 0
     assert bwd(ptr=None) == cp.ERR_ARG
     assert bwd(ws_bytes=need - 1) == cp.ERR_WORKSPACE
     assert bwd(cp_size=0) == cp.ERR_SHAPE

@@ -159,3 +159,40 @@ def test_bwd_accumulate_rejects_mismatched_accumulators(cp):
     with pytest.raises(ValueError):
         cp.bwd_accumulate_(q, q, q, q, lse, q, good, good, good.clone(), 1, True)
     assert cp.launch_count() == n0
+
+
+# chunk lengths that are not multiples of 16 (CUDA-core kernels; any c is allowed)
+ODD = [
+    (1, 2, 96, 64, 2, True, torch.float32),     # c = 24
+    (1, 1, 28, 64, 2, True, torch.float32),     # c = 7
+    (1, 1, 6, 64, 3, True, torch.float32),      # c = 1
+    (1, 2, 40, 128, 5, False, torch.float32),   # c = 8, non-causal
+    (1, 2, 200, 64, 4, True, torch.bfloat16),   # c = 25
+    (2, 1, 120, 128, 3, False, torch.bfloat16), # c = 40
+]
+
+
+@pytest.mark.parametrize("B,H,S,D,cp_size,causal,dtype", ODD)
+def test_any_chunk_length_fwd_bwd_vs_oracle(cp, B, H, S, D, cp_size, causal, dtype):
+    from tests.util import assert_lse_close
+    q, k, v, dout = make_qkv(B, H, S, D, dtype, seed=500 + S + cp_size)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = cp.fwd(qd, kd, vd, cp_size, causal)
+    dq, dk, dv = cp.bwd(qd, kd, vd, o, lse, dod, cp_size, causal)
+    assert cp.sync_status() == cp.OK
+    assert cp.last_path() == 1
+    ro, rl = orc.attn_fwd(np64(q), np64(k), np64(v), causal, D ** -0.5)
+    assert_close(o.cpu(), ro, dtype, "O")
+    assert_lse_close(lse.cpu(), rl)
+    rq, rk, rv = orc.attn_bwd(np64(q), np64(k), np64(v), np64(dout), causal, D ** -0.5)
+    assert_close(dq.cpu(), rq, dtype, "dQ")
+    assert_close(dk.cpu(), rk, dtype, "dK")
+    assert_close(dv.cpu(), rv, dtype, "dV")
+    # the per-step partials merged equal the fused result
+    o_acc = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
+    l_acc = torch.full(q.shape[:-1], float("-inf"), dtype=torch.float32, device="cuda")
+    for t in range(cp_size):
+        op, lp = cp.fwd_step(qd, kd, vd, cp_size, t, causal)
+        cp.merge_(o_acc, l_acc, op, lp)
+    assert cp.sync_status() == cp.OK
+    assert_close(o_acc.cpu(), ro, dtype, "O from steps + merge")

@@ -42,8 +42,8 @@ def test_skipped_load_times_out_and_context_survives(cp):
 
 def test_bad_arguments_do_not_launch(cp):
     n0 = cp.launch_count()
-    q = torch.zeros((1, 1, 100, 128), dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(cp.CpattnError) as e:
+    q = torch.zeros((1, 1, 102, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cp.CpattnError) as e:   # 102 rows are not 4 whole chunks
         cp.fwd(q, q, q, 2, True)
     assert e.value.status == cp.ERR_SHAPE
     q = torch.zeros((1, 1, 256, 128), dtype=torch.float16, device="cuda")

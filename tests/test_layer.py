@@ -68,7 +68,7 @@ def test_layer_rejects_bad_arguments():
         cp.layer_fwd(x, w_qkv, b_qkv, w_o, b_o, 1, 1, True)
     assert e.value.status == cp.ERR_SHAPE
     x, w_qkv, b_qkv, w_o, b_o, _ = (t.cuda() for t in make_layer_inputs(1, 100, 128, seed=1))
-    with pytest.raises(cp.CpattnError) as e:   # S = 100 is not a multiple of 2 * cp_size * 16
+    with pytest.raises(cp.CpattnError) as e:   # B * S = 100 rows: the GEMMs take multiples of 8
         cp.layer_fwd(x, w_qkv, b_qkv, w_o, b_o, 1, 2, True)
     assert e.value.status == cp.ERR_SHAPE
     small = torch.empty(16, dtype=torch.uint8, device="cuda")
