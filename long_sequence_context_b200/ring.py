@@ -9,7 +9,8 @@ rank r + 1; section 5 item 1 -- with a causal mask the sequence is cut into
 note 2 -- the mask is exact.  "Megatron-LM source analysis: Context
 Parallel": section 5 -- the double-buffered loop, the next step's K/V in
 flight while this step's attention runs; section 2 -- the backward mirrors
-the exchange: dK and dV travel around the ring with their K and V.
+the exchange: dK and dV travel around the ring with their K and V (here too
+the running sums of one step are in flight while the next step computes).
 
 Per (q chunk, kv chunk) block the kind follows the same rule as the one-GPU
 path: FULL (kv chunk before the q chunk, or no mask), DIAG (same chunk, masked
@@ -90,6 +91,10 @@ class CudaBlocks:
         self.cp.bwd_accumulate_(q, k, v, o, lse, do, dq_acc, dk_acc, dv_acc, 1, causal=diag,
                                 scale=self.scale, workspace=self._ws)
 
+    def add(self, acc, x):
+        """acc += x, both fp32."""
+        self.cp.accumulate_(acc, x)
+
     def cast(self, acc, dtype):
         return self.cp.finalize(acc, dtype)
 
@@ -121,18 +126,26 @@ def fwd_schedule(rank, world, q, k, v, causal, be):
 
 def bwd_schedule(rank, world, q, k, v, o, lse, do, causal, be):
     """Generator: the backward of rank `rank` from the forward's O and LSE of
-    its rows.  Returns (dq, dk, dv) per own chunk in the inputs' dtype."""
+    its rows.  Returns (dq, dk, dv) per own chunk in the inputs' dtype.
+
+    The dK/dV sums travel around the ring with their K/V.  Step t adds its
+    block terms into fresh sums for the K/V it holds; only then does it take
+    in the running sums of that K/V from rank - 1 (sent at the end of that
+    rank's step t - 1, so in flight during this step's blocks), add them, and
+    send the result on, where it is in flight during step t + 1.  After the
+    last step the sums of this rank's own chunks arrive from rank - 1."""
     own = rank_chunks(rank, world, causal)
     dq = [be.zeros_f32(x) for x in q]
     kv = list(k) + list(v)
-    dkv = [be.zeros_f32(x) for x in kv]  # running dK, dV sums of the chunks in kv
+    pending_dkv = None
     for t in range(world):
         src = (rank - t) % world
         ids = rank_chunks(src, world, causal)
         n = len(ids)
-        pending = None
-        if t + 1 < world:
-            pending = yield ("start", kv)
+        pending_kv = None
+        if t + 1 < world:  # the next step's K/V travels while this step computes
+            pending_kv = yield ("start", kv)
+        dkv = [be.zeros_f32(x) for x in kv]  # this step's dK, dV terms of the K/V held now
         for ai, a in enumerate(own):
             for bi, b in enumerate(ids):
                 kind = block_kind(a, b, causal)
@@ -141,12 +154,15 @@ def bwd_schedule(rank, world, q, k, v, o, lse, do, causal, be):
                 be.bwd_into(q[ai], kv[bi], kv[n + bi], o[ai], lse[ai], do[ai], kind == DIAG,
                             dq[ai], dkv[bi], dkv[n + bi])
         if world > 1:
-            # the sums travel with their K/V; after the last step they reach
-            # the chunks' owner
-            h = yield ("start", dkv)
-            dkv = yield ("finish", h)
+            if t > 0:  # the running sums of the same K/V, from rank - 1
+                incoming = yield ("finish", pending_dkv)
+                for acc, x in zip(dkv, incoming):
+                    be.add(acc, x)
+            pending_dkv = yield ("start", dkv)
         if t + 1 < world:
-            kv = yield ("finish", pending)
+            kv = yield ("finish", pending_kv)
+    if world > 1:
+        dkv = yield ("finish", pending_dkv)
     m = len(own)
     dk = [be.cast(dkv[i], k[i].dtype) for i in range(m)]
     dv = [be.cast(dkv[m + i], v[i].dtype) for i in range(m)]

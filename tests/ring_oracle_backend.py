@@ -62,5 +62,8 @@ class OracleBlocks:
         dk = self.scale * torch.einsum("bhij,bhid->bhjd", ds, q)
         return dq, dk, dv
 
+    def add(self, acc, x):
+        acc += x
+
     def cast(self, acc, dtype):
         return acc.clone()
