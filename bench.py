@@ -802,6 +802,43 @@ def run_ring(args, w):
         dist.destroy_process_group()
 
 
+FP8_METRIC = "causal ring-attn forward on e4m3 inputs TFLOP/s on 1 B200; fraction of the fp8 tensor peak"
+
+
+def run_fp8(args, w):
+    """The e4m3 ring forward alone (inputs quantised before the timed region,
+    as a context-parallel job keeps its K/V in e4m3).  Prints its own JSON line."""
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    from long_sequence_context_b200 import cpattn as cp
+    from long_sequence_context_b200.inputs import workload_inputs
+    peaks = load_peaks()
+    dev = torch.device("cuda", local)
+    q, k, v, _ = workload_inputs(w, with_dout=False)
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    r = time_fp8_fwd(cp, w, qd, kd, vd, peaks, steps=args.steps, warmup=args.warmup)
+    clk = clocks.stop()
+    ms = max_over_ranks(r["ms"], world)
+    if rank == 0:
+        line = {"metric": FP8_METRIC, "value": world * w.flops_fwd() / (ms * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
+                "config": {"workload": f"fp8_{w.name}", "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                           "cp_size": w.cp_size, "causal": w.causal,
+                           "l2": "inputs larger than L2; no flush"},
+                "roofline": r["roofline"], "quantize_ms": r["quantize_ms"],
+                "gpu_launches": int(round(r["launches_per_call"] * args.steps)), "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 MERGE_METRIC = "standalone LSE merge (cpattn_merge) GB/s on 1 B200; fraction of measured HBM copy bandwidth"
 
 
@@ -846,6 +883,8 @@ def main():
                     help="time the multi-rank ring: one sequence split over the --gpus ranks")
     ap.add_argument("--layer", action="store_true",
                     help="time the attention layer (projections + ring attention) instead")
+    ap.add_argument("--fp8", action="store_true",
+                    help="time the e4m3 forward (cpattn_fwd_fp8) alone")
     ap.add_argument("--merge", action="store_true",
                     help="time the standalone LSE merge (cpattn_merge) alone")
     ap.add_argument("--no-extra", action="store_true",
@@ -866,6 +905,8 @@ def main():
         run_reference(args, w)
     elif args.merge:
         run_merge(args)
+    elif args.fp8:
+        run_fp8(args, w)
     elif args.layer:
         run_layer(args, w)
     elif args.ring:

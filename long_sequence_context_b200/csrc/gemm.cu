@@ -9,12 +9,17 @@
 //   dX, dOm  dY W               A K-major,  B MN-major
 //   dW       dY^T X             A MN-major, B MN-major
 //
-// Kernel: persistent, one CTA per SM, 128 x 256 output tiles, k-blocks of 64.
-//   warp 0    TMA producer: A and B k-blocks into a kStages-deep ring (48 KB/stage)
-//   warp 1    MMA issuer (one thread) and TMEM owner: 4 MMAs (M=128, N=256,
-//             K=16) per k-block into one of two 256-column TMEM accumulators
-//   warps 2-5 epilogue: TMEM -> registers (+ bias) -> bf16 -> global memory,
-//             overlapping the next tile's main loop (double-buffered accumulator)
+// Kernel: persistent, one CTA per SM, BM x 256 output tiles, k-blocks of 64.
+//   warp 0    TMA producer: A and B k-blocks into a kStages-deep ring
+//   warp 1    MMA issuer (one thread) and TMEM owner
+//   warps 2.. epilogue: TMEM -> registers (+ bias) -> bf16 -> global memory
+// BM = 128: 4 MMAs (M=128, N=256, K=16) per k-block into one of two 256-column
+//   TMEM accumulators, so four epilogue warps overlap the next tile's main loop
+//   (48 KB per stage, 4 stages).
+// BM = 256: the two 128-row halves of the A tile share each B tile (8 MMAs per
+//   k-block into two 256-column accumulators, 64 KB per stage, 3 stages): a
+//   third less operand traffic per FLOP; eight epilogue warps drain both
+//   halves before the next tile starts.
 // Shared-memory tiles use the 128-byte swizzle.  K-major tiles are rows of 64
 // k-elements (128 B); MN-major tiles are 64-element MN chunks of 64 k-rows,
 // chunk after chunk (the descriptor's leading byte offset is the chunk stride).
@@ -34,17 +39,22 @@ namespace {
 
 using namespace sm100;
 
+template <int BM>
 struct GemmCfg {
-  static constexpr int kBM = 128, kBN = 256, kBK = 64;
-  static constexpr int kStages = 4;
-  static constexpr int kABytes = kBM * kBK * 2;  // 16 KB
-  static constexpr int kBBytes = kBN * kBK * 2;  // 32 KB
+  static constexpr int kBM = BM, kBN = 256, kBK = 64;
+  static constexpr int kHalves = BM / 128;          // 128-row accumulators per tile
+  static constexpr int kStages = BM == 128 ? 4 : 3;
+  static constexpr int kABytes = kBM * kBK * 2;     // 16 / 32 KB
+  static constexpr int kBBytes = kBN * kBK * 2;     // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kChunkBytes = 64 * kBK * 2;  // one MN-major 64 x 64 chunk: 8 KB
   static constexpr int kOffBar = kStages * kStageBytes;
   static constexpr int kSmemBytes = 1024 + kOffBar + 256;
-  static constexpr int kThreads = 192;
-  static constexpr int kGroupM = 8;  // m-blocks per raster group (L2 reuse of B)
+  static constexpr int kEpiWarps = 4 * kHalves;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kAccBufs = BM == 128 ? 2 : 1;  // accumulator sets in TMEM
+  static constexpr int kGroupM = BM == 128 ? 8 : 4;   // m-blocks per raster group (L2 reuse of B)
+  static_assert(kAccBufs * kHalves * kBN == 512, "TMEM columns");
 };
 
 struct GemmParams {
@@ -55,20 +65,21 @@ struct GemmParams {
   unsigned* err;
 };
 
+template <int GROUP_M>
 __device__ __forceinline__ void tile_coords(const GemmParams& P, int t, int& m_blk, int& n_blk) {
-  const int per_group = GemmCfg::kGroupM * P.num_n;
+  const int per_group = GROUP_M * P.num_n;
   const int g = t / per_group, r = t % per_group;
-  const int first_m = g * GemmCfg::kGroupM;
-  const int gm = min(P.num_m - first_m, GemmCfg::kGroupM);
+  const int first_m = g * GROUP_M;
+  const int gm = min(P.num_m - first_m, GROUP_M);
   m_blk = first_m + r % gm;
   n_blk = r / gm;
 }
 
-template <int A_MN, int B_MN>
-__global__ void __launch_bounds__(GemmCfg::kThreads, 1)
+template <int A_MN, int B_MN, int BM>
+__global__ void __launch_bounds__(GemmCfg<BM>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmParams P) {
-  using C = GemmCfg;
+  using C = GemmCfg<BM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -89,7 +100,7 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 128);
+      mbar_init(&acc_empty[i], 32 * C::kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -115,7 +126,7 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
       bool ok = true;
       for (int t = cta; t < P.tiles && ok; t += grid) {
         int mb, nb;
-        tile_coords(P, t, mb, nb);
+        tile_coords<C::kGroupM>(P, t, mb, nb);
         const int m0 = mb * C::kBM, n0 = nb * C::kBN;
         for (int kb = 0; kb < P.nk; ++kb, ++it) {
           const int s = it % C::kStages;
@@ -133,7 +144,7 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
             for (int j = 0; j < C::kBM / 64; ++j)
               tma_load_2d(sA + j * C::kChunkBytes, &tmA, &full[s], m0 + 64 * j, k0);
           } else {
-            tma_load_2d(sA, &tmA, &full[s], k0, m0);
+            tma_load_2d(sA, &tmA, &full[s], k0, m0);  // box: 64 k x BM rows
           }
           if (B_MN) {
 #pragma unroll
@@ -158,7 +169,10 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA --
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(C::kBM, C::kBN, A_MN, B_MN);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::kBN, A_MN, B_MN);
+      // the second 128-row half of A: 128 rows of 128 B further (K-major), or
+      // two 64-row MN chunks further (MN-major) -- 16 KB either way
+      constexpr uint32_t kHalfA = 16384;
       // K-major: 16 k-elements = 32 bytes along the swizzled row; MN-major: 16
       // k-rows = 2048 bytes (two 8-row groups of 128 B)
       constexpr uint32_t kStepA = A_MN ? 2048 : 32, kStepB = B_MN ? 2048 : 32;
@@ -166,10 +180,11 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
       uint32_t it = 0, lt = 0;
       bool ok = true;
       for (int t = cta; t < P.tiles && ok; t += grid, ++lt) {
-        const uint32_t acc = lt & 1;
-        if (lt >= 2 && !mbar_wait(&acc_empty[acc], ((lt >> 1) - 1) & 1, abort_flag, P.err)) break;
+        const uint32_t acc = C::kAccBufs == 2 ? (lt & 1) : 0;
+        const uint32_t use = C::kAccBufs == 2 ? (lt >> 1) : lt;  // earlier uses of this set
+        if (use >= 1 && !mbar_wait(&acc_empty[acc], (use - 1) & 1, abort_flag, P.err)) break;
         tc_fence_after();
-        const uint32_t tacc = tmem_base + acc * C::kBN;
+        const uint32_t tacc = tmem_base + acc * C::kHalves * C::kBN;
         for (int kb = 0; kb < P.nk; ++kb, ++it) {
           const int s = it % C::kStages;
           if (!mbar_wait(&full[s], (it / C::kStages) & 1, abort_flag, P.err)) {
@@ -182,8 +197,10 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
           const uint64_t dB = smem_desc_sw128(aA + C::kABytes, lboB, 1024);
 #pragma unroll
           for (int kk = 0; kk < C::kBK / 16; ++kk)
-            mma_ss(tacc, desc_at(dA, kk * kStepA), desc_at(dB, kk * kStepB), idesc,
-                   (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h)
+              mma_ss(tacc + h * C::kBN, desc_at(dA, h * kHalfA + kk * kStepA),
+                     desc_at(dB, kk * kStepB), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
         }
         if (!ok) break;
@@ -197,18 +214,22 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
     __syncwarp();
   } else {
     // -------------------------------------------------------- epilogue --
-    const int quarter = warp & 3;  // warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
+    // warps 2..5 -> TMEM lane quarters 2, 3, 0, 1 of the first 128-row half,
+    // warps 6..9 (BM = 256) the same quarters of the second half
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     uint32_t lt = 0;
     for (int t = cta; t < P.tiles; t += grid, ++lt) {
-      const uint32_t acc = lt & 1;
-      if (!mbar_wait_warp(&acc_full[acc], (lt >> 1) & 1, abort_flag, P.err)) break;
+      const uint32_t acc = C::kAccBufs == 2 ? (lt & 1) : 0;
+      const uint32_t use = C::kAccBufs == 2 ? (lt >> 1) : lt;
+      if (!mbar_wait_warp(&acc_full[acc], use & 1, abort_flag, P.err)) break;
       tc_fence_after();
       int mb, nb;
-      tile_coords(P, t, mb, nb);
-      const int row = mb * C::kBM + quarter * 32 + lane;
+      tile_coords<C::kGroupM>(P, t, mb, nb);
+      const int row = mb * C::kBM + half * 128 + quarter * 32 + lane;
       const int n0 = nb * C::kBN;
-      const uint32_t tacc = tmem_base + lane_off + acc * C::kBN;
+      const uint32_t tacc = tmem_base + lane_off + (acc * C::kHalves + half) * C::kBN;
 #pragma unroll 1
       for (int cb = 0; cb < C::kBN; cb += 32) {
         if (n0 + cb >= P.N) break;  // warp-uniform
@@ -253,10 +274,10 @@ __global__ void __launch_bounds__(GemmCfg::kThreads, 1)
   }
 }
 
-template <int A_MN, int B_MN>
+template <int A_MN, int B_MN, int BM>
 int launch(const void* A, const void* B, const void* bias, void* Cm, int M, int N, int K,
            unsigned* err, cudaStream_t stream) {
-  using C = GemmCfg;
+  using C = GemmCfg<BM>;
   CUtensorMap ta, tb;
   // A: K-major [M][K] (box 64 k x 128 rows) or MN-major [K][M] (box 64 m x 64 k)
   const bool okA = A_MN ? make_tmap_bf16_2d(&ta, A, K, M, 64, 64)
@@ -276,13 +297,13 @@ int launch(const void* A, const void* B, const void* bias, void* Cm, int M, int 
   P.bias = static_cast<const __nv_bfloat16*>(bias);
   P.err = err;
   static std::atomic<unsigned long long> attr_done{0};
-  if (!smem_attr_once(gemm_kernel<A_MN, B_MN>, C::kSmemBytes, attr_done)) return -1;
+  if (!smem_attr_once(gemm_kernel<A_MN, B_MN, BM>, C::kSmemBytes, attr_done)) return -1;
   int dev = 0;
   cudaGetDevice(&dev);
   int grid = num_sms(dev);
   if (grid > P.tiles) grid = P.tiles;
   prof_begin(kKGemm, stream);
-  gemm_kernel<A_MN, B_MN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(ta, tb, P);
+  gemm_kernel<A_MN, B_MN, BM><<<grid, C::kThreads, C::kSmemBytes, stream>>>(ta, tb, P);
   prof_end(kKGemm, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
@@ -298,12 +319,16 @@ int gemm_check(int M, int N, int K) {
   return 0;
 }
 
+// 128-row tiles (kGemmBM = 128) or 256-row tiles (256)
+constexpr int kGemmBM = 256;
+
 int launch_gemm(const void* A, const void* B, const void* bias, void* C, int M, int N, int K,
                 int a_mn, int b_mn, unsigned* err, cudaStream_t stream) {
-  if (a_mn && b_mn) return launch<1, 1>(A, B, bias, C, M, N, K, err, stream);
-  if (a_mn) return launch<1, 0>(A, B, bias, C, M, N, K, err, stream);
-  if (b_mn) return launch<0, 1>(A, B, bias, C, M, N, K, err, stream);
-  return launch<0, 0>(A, B, bias, C, M, N, K, err, stream);
+  constexpr int BM = kGemmBM;
+  if (a_mn && b_mn) return launch<1, 1, BM>(A, B, bias, C, M, N, K, err, stream);
+  if (a_mn) return launch<1, 0, BM>(A, B, bias, C, M, N, K, err, stream);
+  if (b_mn) return launch<0, 1, BM>(A, B, bias, C, M, N, K, err, stream);
+  return launch<0, 0, BM>(A, B, bias, C, M, N, K, err, stream);
 }
 
 }  // namespace cpattn
