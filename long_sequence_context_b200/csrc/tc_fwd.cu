@@ -55,24 +55,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kRescaleThresholdF8 = 2.0f;
 constexpr float kP8Log2Scale = 6.0f;  // e4m3 P holds 2^6 * P
-// e4m3 softmax: of every four exponentials, this many are evaluated on the FMA
-// pipe (ex2_fma) instead of the special-function unit, which the e4m3 kernel
-// otherwise saturates (its products take half the tensor time of bf16 ones)
-constexpr int kFmaExpPer4 = 1;
-
-// 2^x on the FMA pipe: x = n + f with n = floor(x), f in [0, 1); 2^f from the
-// cubic that interpolates it at the four Chebyshev nodes of [0, 1] (relative
-// error < 1.0e-4, far below e4m3's 2^-4 rounding of P), 2^n added to the
-// exponent field.  Arguments below -126 give 0 (masked scores are -inf).
-__device__ __forceinline__ float ex2_fma(float x) {
-  const float xc = fmaxf(x, -126.f);
-  const float fl = floorf(xc);
-  const float f = xc - fl;
-  const float p = fmaf(fmaf(fmaf(0.07896725704217157f, f, 0.2246931557639988f), f,
-                            0.6963247710915813f), f, 0.9999002881727679f);
-  const float r = __int_as_float(__float_as_int(p) + ((int)fl << 23));
-  return x < -126.f ? 0.f : r;
-}
 
 template <int D, bool F8>
 struct FwdCfg {
@@ -82,8 +64,10 @@ struct FwdCfg {
   static constexpr int kSubBytes = kTile * 128;           // one 128-byte-wide swizzled block
   static constexpr int kStages = F8 ? 10 : (D == 128 ? 5 : 8);  // K/V slots
   static constexpr int kThreads = 384;
-  static constexpr int kRegsSoftmax = 208;  // 2*128*208 + 128*80 <= 384*168
-  static constexpr int kRegsOther = 80;
+  // setmaxnreg split of the 384 x 168 launch registers: 2*128*Rs + 128*Ro <= 64512
+  // (e4m3: 216 / 72 leaves the packed softmax free of spills)
+  static constexpr int kRegsSoftmax = F8 ? 216 : 208;
+  static constexpr int kRegsOther = F8 ? 72 : 80;
   static constexpr int kBarOffset = 2 * kTileBytes + kStages * kTileBytes;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
   static constexpr uint32_t kIdescQK = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, 0, 0);
@@ -327,10 +311,7 @@ __global__ void __launch_bounds__(384, 1)
             const float x1 = fmaf(__uint_as_float(r[c + 1]), sl2, -base);
             const float x2 = fmaf(__uint_as_float(r[c + 2]), sl2, -base);
             const float x3 = fmaf(__uint_as_float(r[c + 3]), sl2, -base);
-            const float p0 = ex2(x0);
-            const float p1 = kFmaExpPer4 >= 3 ? ex2_fma(x1) : ex2(x1);
-            const float p2 = kFmaExpPer4 >= 2 ? ex2_fma(x2) : ex2(x2);
-            const float p3 = kFmaExpPer4 >= 1 ? ex2_fma(x3) : ex2(x3);
+            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
             ls[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
             r[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);  // r[c/4] was read at or before this step
           }
