@@ -179,11 +179,6 @@ __global__ void __launch_bounds__(GemmCfg<BM>::kThreads, 1)
       constexpr uint32_t lboA = A_MN ? C::kChunkBytes : 16, lboB = B_MN ? C::kChunkBytes : 16;
       uint32_t it = 0, lt = 0;
       bool ok = true;
-      // The barrier of the next k-block is tested between the MMAs of the
-      // current one (a test between MMA groups leaves the tensor pipe idle; one
-      // between two MMAs of a group costs little), and waited on only if that
-      // test did not already see the stage full.
-      Probe pr;
       for (int t = cta; t < P.tiles && ok; t += grid, ++lt) {
         const uint32_t acc = C::kAccBufs == 2 ? (lt & 1) : 0;
         const uint32_t use = C::kAccBufs == 2 ? (lt >> 1) : lt;  // earlier uses of this set
@@ -192,24 +187,20 @@ __global__ void __launch_bounds__(GemmCfg<BM>::kThreads, 1)
         const uint32_t tacc = tmem_base + acc * C::kHalves * C::kBN;
         for (int kb = 0; kb < P.nk; ++kb, ++it) {
           const int s = it % C::kStages;
-          if (kb == 0) pr.set(&full[s], (it / C::kStages) & 1);
-          if (!pr.finish(abort_flag, P.err)) {
+          if (!mbar_wait(&full[s], (it / C::kStages) & 1, abort_flag, P.err)) {
             ok = false;
             break;
           }
-          if (kb + 1 < P.nk) pr.set(&full[(it + 1) % C::kStages], ((it + 1) / C::kStages) & 1);
           tc_fence_after();
           const uint32_t aA = smem_u32(smem + s * C::kStageBytes);
           const uint64_t dA = smem_desc_sw128(aA, lboA, 1024);
           const uint64_t dB = smem_desc_sw128(aA + C::kABytes, lboB, 1024);
 #pragma unroll
-          for (int kk = 0; kk < C::kBK / 16; ++kk) {
+          for (int kk = 0; kk < C::kBK / 16; ++kk)
 #pragma unroll
             for (int h = 0; h < C::kHalves; ++h)
               mma_ss(tacc + h * C::kBN, desc_at(dA, h * kHalfA + kk * kStepA),
                      desc_at(dB, kk * kStepB), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-            if (kk == 1 || kk == 3) pr.test();
-          }
           tc_commit(&empty[s]);
         }
         if (!ok) break;

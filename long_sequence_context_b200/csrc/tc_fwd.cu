@@ -1,8 +1,8 @@
 // tc_fwd.cu -- tcgen05 tensor-core ring-attention forward for bf16, D in {64,128}.
 //
-// One persistent kernel runs every virtual rank and every ring step.  A work
-// item is a pair of 128-row Q tiles of one chunk; its K/V tiles are walked in
-// ring order (step t: the chunks of rank (r - t) mod N, SKIP blocks never
+// One kernel runs every virtual rank and every ring step.  A work item (one
+// CTA, longest items first) is a pair of 128-row Q tiles of one chunk; its K/V
+// tiles are walked in ring order (step t: the chunks of rank (r - t) mod N, SKIP blocks never
 // visited, DIAG blocks stopping at the pair's diagonal), and the per-step
 // partials are merged on chip by the online log-sum-exp rescale.  Sources:
 // "Configuring RingAttention+FlashAttention for CP" (devpress.csdn.net),
@@ -627,10 +627,13 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   P.stall = stall;
   static std::atomic<unsigned long long> attr_done{0};
   if (!smem_attr_once(tc_fwd_kernel<D, F8>, C::kSmemBytes, attr_done)) return -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  int grid = num_sms(dev);
-  if (grid > P.n_items) grid = P.n_items;
+  // One CTA per work item, items numbered longest first (heads four at a
+  // time): the hardware block scheduler hands them out in that order as SMs
+  // free up, a greedy longest-first schedule.  A persistent grid with a static
+  // snake assignment of the same order measured 4% slower at S = 32K and
+  // balances far worse on small problems (S = 8K: a third of the SMs idle at
+  // the end).
+  const int grid = P.n_items;
   const int prof_id = F8 ? kKTcFwdFp8 : kKTcFwd;
   prof_begin(prof_id, stream);
   tc_fwd_kernel<D, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, P);
