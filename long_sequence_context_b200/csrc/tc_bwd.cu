@@ -22,10 +22,14 @@
 // fp32 dQ reduction traffic, which on this GPU costs more than the extra
 // tensor work.
 //
-// dK / dV kernel: one CTA per K/V tile, 320 threads.  Warps 0-7 do the elementwise work:
+// dK / dV kernel: one CTA per K/V tile, 384 threads.  Warps 0-7 do the elementwise work:
 // warp w owns TMEM lanes 32*(w%4).. (one key row per thread) and the column
 // half w/4 of each 128-column score tile.  Warp 8 issues TMA loads, warp 9 the
-// MMAs (one thread) and owns TMEM.  The bf16 P^T / dS^T values of a column half
+// MMAs (one thread) and owns TMEM; warps 10-11 only complete the third
+// warpgroup, whose registers go to the elementwise warps (setmaxnreg 208 / 88:
+// with 320 threads every thread would be capped at 168, two warps short of a
+// warpgroup on two of the four SM sub-partitions; measured 16.4 against
+// 16.9 ms).  The bf16 P^T / dS^T values of a column half
 // are packed into the first half of that half's own TMEM columns (half 0 ->
 // columns [0,32), half 1 -> [64,96)), so neither half overwrites scores the
 // other is still reading; the MMA k-steps address them accordingly.
@@ -79,7 +83,7 @@ struct DkdvCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     tc_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                    const BwdParams P) {
@@ -140,6 +144,7 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp < 8) {
     // ---------------------------------------------------- P^T and dS^T --
+    regs_inc<208>();
     const int quarter = warp & 3, half = warp >> 2;
     const int rloc = quarter * 32 + lane;  // key row within the K/V tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -244,7 +249,10 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(acc_free);
     }
-  } else if (warp == 8) {
+  } else {
+    regs_dec<88>();
+  }
+  if (warp == 8) {
     // ----------------------------------------------------------------- TMA --
     uint32_t items = 0, q_cnt = 0;
     bool ok = true;
@@ -305,7 +313,7 @@ __global__ void __launch_bounds__(320, 1)
                globaltimer() - t0 < kWaitLimitNs) {
         }
     }
-  } else {
+  } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
     // One thread issues every MMA (the other lanes wait at the end).  The
     // tensor pipe queues very few MMAs ahead of it, so a barrier wait between
@@ -494,7 +502,7 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   // 1-2% slower here.)
   const int grid = P.n_items;
   prof_begin(kKTcDkdv, stream);
-  tc_dkdv_kernel<D><<<grid, 320, DkdvCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
+  tc_dkdv_kernel<D><<<grid, 384, DkdvCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
   prof_end(kKTcDkdv, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
   if (launch_tc_dq<D>(P, mq, mk, mv, mdo, grid, stream) < 0) return -1;
