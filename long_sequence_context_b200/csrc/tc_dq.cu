@@ -16,9 +16,11 @@
 // the tensor core is busy while the elementwise warps work.
 //
 // TMEM (512 columns): S0 [0,128) S1 [128,256) dP [256,384) dQ [384,384+D).
-// Roles (320 threads): warps 0-7 elementwise (warp w: TMEM lanes 32*(w%4)..,
-// score columns 64*(w/4)..), warp 8 TMA (Q, dO per item; a ring of K / V
-// tiles), warp 9 MMA issuer and TMEM owner.  dS of column half h is packed as
+// Roles (384 threads): warps 0-7 elementwise (warp w: TMEM lanes 32*(w%4)..,
+// score columns 64*(w/4)..; 208 registers via setmaxnreg), warp 8 TMA (Q, dO
+// per item; a ring of K / V tiles), warp 9 MMA issuer and TMEM owner, warps
+// 10-11 only complete the third warpgroup (88 registers).  One CTA per Q tile,
+// longest first.  dS of column half h is packed as
 // bf16 into columns [64 h, 64 h + 32) of its S buffer.
 // Sources: "Configuring RingAttention+FlashAttention for CP", section 3 code and
 // note 2, section 5 item 1 (ring walk, mask, zigzag); the gradient is that of
@@ -63,7 +65,7 @@ __device__ __forceinline__ uint32_t packed_col(int c) { return (c & 64) + ((c & 
 __device__ __forceinline__ uint32_t packed_kstep(int kk) { return (kk >= 4 ? 64 : 0) + (kk & 3) * 8; }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     tc_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                  const BwdParams P) {
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp < 8) {
     // ---------------------------------------------------------- elementwise --
+    regs_inc<208>();
     const int quarter = warp & 3, half = warp >> 2;
     const int rloc = quarter * 32 + lane;  // query row within the Q tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -197,7 +200,10 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(acc_free);
     }
-  } else if (warp == 8) {
+  } else {
+    regs_dec<88>();
+  }
+  if (warp == 8) {
     // ----------------------------------------------------------------- TMA --
     uint32_t kv_idx = 0, items = 0;
     bool ok = true;
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(320, 1)
                globaltimer() - t0 < kWaitLimitNs) {
         }
     }
-  } else {
+  } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
     const uint32_t tDP = tmem_base + C::kColDP, tDQ = tmem_base + C::kColDQ;
     const uint32_t aQ = smem_u32(sQ), adO = smem_u32(sdO), aKV = smem_u32(sKV);
@@ -396,7 +402,7 @@ int launch_tc_dq(const BwdParams& P, const CUtensorMap& mq, const CUtensorMap& m
   static std::atomic<unsigned long long> attr_done{0};
   if (!smem_attr_once(tc_dq_kernel<D>, C::kSmemBytes, attr_done)) return -1;
   prof_begin(kKTcDq, stream);
-  tc_dq_kernel<D><<<grid, 320, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
+  tc_dq_kernel<D><<<grid, 384, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
   prof_end(kKTcDq, stream);
   return cudaGetLastError() == cudaSuccess ? 1 : -1;
 }
