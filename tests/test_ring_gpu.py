@@ -20,6 +20,7 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("world,causal,S", [
     (2, True, 1024),    # chunks of 256: tcgen05 blocks
     (4, True, 1024),    # chunks of 128: DIAG blocks on the CUDA-core kernels
+    (3, True, 1536),    # an odd ring: the dK/dV sums make three hops
     (2, False, 1024),
 ])
 def test_loopback_ring_with_library_blocks(world, causal, S):
