@@ -25,3 +25,14 @@ def test_digest_covers_the_listed_sources():
     d = bench.kernel_source_digest("tc_dkdv")
     assert len(d) == 64 and d == bench.kernel_source_digest("tc_dkdv")
     assert "tc_bwd.cu" in bench.KERNEL_SOURCES["tc_dkdv"]
+
+
+def test_committed_traffic_record_matches_the_current_sources():
+    # the committed capture describes the kernel as it is in the tree
+    assert bench.recorded_traffic("tc_dkdv", "causal_b1h32s32768d128_cp8_bf16") is not None
+
+
+def test_merge_bytes_per_row():
+    # read acc O + LSE, read part O + LSE, write acc O + LSE (fp32)
+    assert bench.merge_bytes_per_row(128) == 1548
+    assert bench.merge_bytes_per_row(64) == 3 * 64 * 4 + 12
