@@ -63,9 +63,10 @@ def test_amax_is_exact(cp, dtype):
         assert a.item() == np.float32(np.abs(_f32(t)).max())
 
 
-@pytest.mark.parametrize("B,H,S,D", [(1, 2, 1024, 128), (2, 3, 256, 64), (1, 4, 8192, 128)])
-def test_quantize_matches_oracle_codes_bitwise(cp, B, H, S, D):
-    q, _, v, _ = make_qkv(B, H, S, D, torch.bfloat16, seed=62 + S)
+@pytest.mark.parametrize("B,H,S,D,dtype", [(1, 2, 1024, 128, torch.bfloat16), (2, 3, 256, 64, torch.bfloat16),
+                                           (1, 4, 8192, 128, torch.bfloat16), (1, 2, 512, 128, torch.float32)])
+def test_quantize_matches_oracle_codes_bitwise(cp, B, H, S, D, dtype):
+    q, _, v, _ = make_qkv(B, H, S, D, dtype, seed=62 + S)
     for x, transpose in ((q, False), (v, True)):
         xd = x.cuda()
         a = cp.amax(xd)
@@ -153,3 +154,28 @@ def test_fwd_fp8_rejects_unsupported_shapes(cp):
         cp.fwd_fp8(z, z, zt, a3, 2, True)
     assert e.value.status == cp.ERR_SHAPE
     assert cp.sync_status() == cp.OK
+
+
+def test_fp8_all_zero_values_and_tiny_inputs(cp):
+    """An all-zero V (max|v| = 0: scale 1, every code 0) gives O = 0 exactly;
+    inputs a million times smaller than N(0, 1) quantise to the same codes as
+    the unit-scale ones (the per-tensor scale absorbs the magnitude) and give
+    the oracle's result within the same bound."""
+    B, H, S, D, cp_size = 1, 2, 1024, 128, 2
+    q, k, v, _ = make_qkv(B, H, S, D, torch.bfloat16, seed=81)
+    zero = torch.zeros_like(v).cuda()
+    q8, k8, vt8, a3 = cp.quantize_qkv_e4m3(q.cuda(), k.cuda(), zero)
+    o, lse = cp.fwd_fp8(q8, k8, vt8, a3, cp_size, True)
+    assert cp.sync_status() == cp.OK
+    assert a3[2].item() == 0.0
+    assert int(vt8.count_nonzero().item()) == 0
+    assert torch.count_nonzero(o).item() == 0 and torch.isfinite(lse).all()
+    tiny = [(t.float() * 1e-6).to(torch.bfloat16) for t in (q, k, v)]
+    q8t, k8t, vt8t, a3t = cp.quantize_qkv_e4m3(*(t.cuda() for t in tiny))
+    want, _, _ = oracle_quantized(tiny[0])
+    assert np.array_equal(q8t.cpu().numpy(), want)
+    o, lse = cp.fwd_fp8(q8t, k8t, vt8t, a3t, cp_size, True, scale=D ** -0.5 * 1e12)
+    assert cp.sync_status() == cp.OK
+    (_, qd, _), (_, kd, _), (_, vd, _) = (oracle_quantized(t) for t in tiny)
+    check_rows(cp, o.float() * 1e6, lse, qd, kd, vd * 1e6, True, D ** -0.5 * 1e12, [(0, 0), (0, 1)],
+               lambda b, h: np.arange(S))
