@@ -54,14 +54,31 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// The waits below take the barrier's 32-bit shared-window address.
+__device__ __forceinline__ bool mbar_try_wait_at(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait_at(smem_u32(bar), parity);
+}
+
+// Non-blocking test of phase `parity` (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_at(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -69,13 +86,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for phase `parity` of `bar`.  Returns false when the CTA-wide
 // abort flag is already raised or the wait ran out; in the second case it
 // raises the flag and records kErrTimeout in the device error word.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait_at(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned* err) {
+  if (mbar_try_wait_at(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (*abort_flag) return false;
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_at(bar, parity)) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
       atomicOr(err, kErrTimeout);
@@ -83,28 +100,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
   }
 }
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned* err) {
+  return mbar_wait_at(smem_u32(bar), parity, abort_flag, err);
+}
 
 // A barrier test whose result is needed only later.  The thread that issues
 // MMAs tests the barrier of its next group between two MMAs of the current
 // one: the test's latency then overlaps queued tensor work instead of leaving
 // the tensor pipe idle between groups (the pipe queues very few MMAs ahead of
-// the issuing thread).
+// the issuing thread).  The test never suspends the thread.
 struct Probe {
-  uint64_t* bar = nullptr;  // nullptr: nothing to test
+  uint32_t bar = 0;  // shared-window address; 0: nothing to test
   uint32_t parity = 0;
   bool done = true;
   __device__ __forceinline__ void set(uint64_t* b, uint32_t p) {
-    bar = b;
+    bar = smem_u32(b);
     parity = p;
     done = false;
   }
   __device__ __forceinline__ void test() {
-    if (bar != nullptr && !done) done = mbar_try_wait(bar, parity);
+    if (!done) done = mbar_test_at(bar, parity);
   }
   // complete the wait if the early test did not see the phase finished
   __device__ __forceinline__ bool finish(volatile int* abort_flag, unsigned* err) {
-    const bool r = done || mbar_wait(bar, parity, abort_flag, err);
-    bar = nullptr;
+    const bool r = done || mbar_wait_at(bar, parity, abort_flag, err);
     done = true;
     return r;
   }
@@ -371,6 +391,47 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+// Packed fp32 pairs: one instruction computes both lanes, each rounded as the
+// scalar operation would be.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, C, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mov.b64 C, {%6, %7};\n\tfma.rn.f32x2 D, A, B, C;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "add.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "sub.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mul.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// max of three (one instruction)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ float ex2(float x) {

@@ -14,25 +14,29 @@
 //   1. preprocess: delta_i = rowsum(dO_i * O_i), LSE_i * log2(e)   (workspace)
 //   2. dK / dV kernel: one 128-key K/V tile per work item; walks the q tiles
 //      that see it in mirror ring order (at step t the K/V of rank `owner` sits
-//      on rank owner + t): S^T = K Q^T, dP^T = V dO^T (TMEM), P^T and dS^T
-//      (bf16, back into TMEM), dV += P^T dO, dK += dS^T Q (A from TMEM).
+//      on rank owner + t): S^T = K Q^T, dP^T = V dO^T (TMEM), P^T (bf16, to
+//      shared memory) and dS^T (bf16, back into TMEM), dV += P^T dO,
+//      dK += dS^T Q (A from TMEM).
 //   3. dQ kernel (tc_dq.cu): one Q tile per work item, dQ accumulated in TMEM
 //      and written once; no reductions.
 // Computing dQ in its own kernel recomputes S and dP once more but removes the
 // fp32 dQ reduction traffic, which on this GPU costs more than the extra
 // tensor work.
 //
-// dK / dV kernel: one CTA per K/V tile, 384 threads.  Warps 0-7 do the elementwise work:
-// warp w owns TMEM lanes 32*(w%4).. (one key row per thread) and the column
-// half w/4 of each 128-column score tile.  Warp 8 issues TMA loads, warp 9 the
-// MMAs (one thread) and owns TMEM; warps 10-11 only complete the third
-// warpgroup, whose registers go to the elementwise warps (setmaxnreg 208 / 88:
-// with 320 threads every thread would be capped at 168, two warps short of a
-// warpgroup on two of the four SM sub-partitions; measured 16.4 against
-// 16.9 ms).  The bf16 P^T / dS^T values of a column half
-// are packed into the first half of that half's own TMEM columns (half 0 ->
-// columns [0,32), half 1 -> [64,96)), so neither half overwrites scores the
-// other is still reading; the MMA k-steps address them accordingly.
+// dK / dV kernel: one CTA per K/V tile, 384 threads.  Warps 0-7 do the
+// elementwise work: warp w owns TMEM lanes 32*(w%4).. (one key row per thread)
+// and the column half w/4 of each 128-column score tile.  Warp 8 issues TMA
+// loads, warp 9 the MMAs (one thread) and owns TMEM; warps 10-11 only complete
+// the third warpgroup (setmaxnreg: 200 registers for the elementwise warps,
+// 104 for the rest; 384 x 168 at launch).
+// TMEM (512 columns): S^T [0,128) dP^T [128,256) dV [256,256+D) dK [384,384+D)
+// (D = 64: dK at 320).  The elementwise warps read S^T out of TMEM at once and
+// release it, so the next q tile's S^T is computed during their exponential
+// phase; P^T goes to shared memory (the A operand of dV += P^T dO, K-major,
+// 128-byte swizzle) and dS^T back into dP^T's columns, packed: column half h
+// into [128 + 64 h, 128 + 64 h + 32), so neither half overwrites values the
+// other is still reading.  The MMA thread tests the barriers of its next MMA
+// group between the MMAs of the current one.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -74,12 +78,20 @@ struct DkdvCfg {
   static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr int kOffLD = kOffQ + kStages * 2 * kTileBytes;  // stage s: LSE2[128], delta[128]
   static constexpr int kLDBytes = 1024;
-  static constexpr int kOffBar = kOffLD + kStages * kLDBytes;
-  static constexpr int kSmemBytes = 1024 + kOffBar + 256;
+  // P^T of the current q tile, bf16 [128 keys][128 q] as two 64-column swizzled
+  // blocks: the A operand (K-major) of dV += P^T dO
+  static constexpr int kOffP = kOffLD + kStages * kLDBytes;
+  static constexpr int kDataBytes = kOffP + 128 * 128 * 2;
+  static constexpr int kBarBytes = 256;
+  // the barriers sit in the alignment slack in front of the 1024-aligned data
+  // when it has room for them, else behind the data
+  static constexpr int kSmemBytes = 1024 + kDataBytes;
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
   static constexpr uint32_t kColDK = (D == 128) ? 384 : 320;
   static constexpr uint32_t kIdescST = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 0, 1);
+  static_assert(kOffP % 1024 == 0, "swizzled P^T blocks need 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 template <int D>
@@ -91,21 +103,29 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
+  // (chosen on the 32-bit shared-window address, so that the barrier
+  // addresses stay constant offsets of one 32-bit base)
+  const uint32_t raw_s = smem_u32(smem_raw), data_s = smem_u32(smem);
+  const uint32_t bar_s = (data_s - raw_s >= (uint32_t)C::kBarBytes) ? raw_s : data_s + C::kDataBytes;
+  uint8_t* bar_area = static_cast<uint8_t*>(__cvta_shared_to_generic(bar_s));
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint8_t* sP = smem + C::kOffP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
   uint64_t* q_full = bars + 2;             // [kStages]
   uint64_t* q_empty = q_full + C::kStages;  // [kStages]
   uint64_t* s_ready = q_empty + C::kStages;  // S^T of the q tile in TMEM
   uint64_t* dp_ready = s_ready + 1;          // dP^T of the q tile in TMEM
-  uint64_t* pa_ready = s_ready + 2;          // P^T written back (256 arrivals)
+  uint64_t* pa_ready = s_ready + 2;          // P^T in shared memory (256 arrivals)
   uint64_t* pb_ready = s_ready + 3;          // dS^T written back (256 arrivals)
   uint64_t* kv_done = s_ready + 4;
   uint64_t* acc_free = s_ready + 5;
   uint64_t* drain = s_ready + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_ready + 7);
+  uint64_t* s_free = s_ready + 7;            // S^T read out of TMEM (256 arrivals)
+  uint64_t* p_free = s_ready + 8;            // dV MMA done reading P^T
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_ready + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,6 +143,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(kv_done, 1);
     mbar_init(acc_free, 256);
     mbar_init(drain, 1);
+    mbar_init(s_free, 256);
+    mbar_init(p_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -144,12 +166,14 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp < 8) {
     // ---------------------------------------------------- P^T and dS^T --
-    regs_inc<208>();
+    regs_inc<200>();
     const int quarter = warp & 3, half = warp >> 2;
     const int rloc = quarter * 32 + lane;  // key row within the K/V tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem_base + lane_off + C::kColS;
     const uint32_t tDP = tmem_base + lane_off + C::kColDP;
+    // this thread's 128-byte row of P^T: key rloc, q columns [64 half, 64 half + 64)
+    uint8_t* prow = sP + half * C::kSubBytes + rloc * 128;
     uint32_t s_cnt = 0, items = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
@@ -162,60 +186,80 @@ __global__ void __launch_bounds__(384, 1)
       int qt, dg;
       while (qi.next(P, qt, dg)) {
         const int st = s_cnt % C::kStages;
-        // exponential phase: needs S^T only; P^T goes back to TMEM for dV
+        // exponential phase: S^T is read out of TMEM at once (the next q tile's
+        // S^T may then be computed into the same columns); P^T goes to shared
+        // memory for dV
         if (!mbar_wait_warp(s_ready, s_cnt & 1, abort_flag, P.err) ||
             !mbar_wait_warp(&q_full[st], (s_cnt / C::kStages) & 1, abort_flag, P.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        uint32_t sv[64];
+        tmem_ld32<0>(tS + half * 64, sv);
+        tmem_ld32<32>(tS + half * 64 + 32, sv);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_free);
         const float4* l4 = reinterpret_cast<const float4*>(smem + C::kOffLD + st * C::kLDBytes);
         const float4* d4 = l4 + 32;
         float p[64];
+        const float2 sl = make_float2(P.sl2, P.sl2);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const int cb = half * 64 + ch * 32;  // first q column of this chunk
-          uint32_t sv[32], pk[16];
-          tmem_ld32<0>(tS + cb, sv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 L = l4[(cb >> 2) + c4];
-            const float lv[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float pe = ex2(fmaf(__uint_as_float(sv[4 * c4 + e]), P.sl2, -lv[e]));
-              if (dg && rloc > cb + 4 * c4 + e) pe = 0.f;  // key after query: masked
-              p[ch * 32 + 4 * c4 + e] = pe;
-            }
-            pk[2 * c4] = pack_bf16x2(p[ch * 32 + 4 * c4], p[ch * 32 + 4 * c4 + 1]);
-            pk[2 * c4 + 1] = pack_bf16x2(p[ch * 32 + 4 * c4 + 2], p[ch * 32 + 4 * c4 + 3]);
-          }
-          tmem_st16<0>(tS + packed_col(cb), pk);
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 L = l4[half * 16 + c4];
+          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[4 * c4]), __uint_as_float(sv[4 * c4 + 1])), sl,
+                                   make_float2(-L.x, -L.y));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[4 * c4 + 2]), __uint_as_float(sv[4 * c4 + 3])), sl,
+                                   make_float2(-L.z, -L.w));
+          p[4 * c4 + 0] = ex2(x01.x);
+          p[4 * c4 + 1] = ex2(x01.y);
+          p[4 * c4 + 2] = ex2(x23.x);
+          p[4 * c4 + 3] = ex2(x23.y);
         }
-        tmem_wait_st();
-        tc_fence_before();
+        if (dg) {
+          // diagonal tile: keys after the query are masked
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (rloc > half * 64 + c) p[c] = 0.f;
+        }
+        // the previous q tile's dV MMA must be done reading P^T
+        if (s_cnt > 0 && !mbar_wait_warp(p_free, (s_cnt - 1) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 u = make_uint4(pack_bf16x2(p[8 * ch], p[8 * ch + 1]), pack_bf16x2(p[8 * ch + 2], p[8 * ch + 3]),
+                                     pack_bf16x2(p[8 * ch + 4], p[8 * ch + 5]), pack_bf16x2(p[8 * ch + 6], p[8 * ch + 7]));
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (rloc & 7)) << 4)) = u;
+        }
+        fence_proxy_async_smem();
         mbar_arrive(pa_ready);
         // dS phase: needs dP^T; dS^T goes back to TMEM for dK
         if (!mbar_wait_warp(dp_ready, s_cnt & 1, abort_flag, P.err)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
+        uint32_t dpv[64];
+        tmem_ld32<0>(tDP + half * 64, dpv);
+        tmem_ld32<32>(tDP + half * 64 + 32, dpv);
+        tmem_wait_ld();
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           const int cb = half * 64 + ch * 32;
-          uint32_t dpv[32], dsk[16];
-          tmem_ld32<0>(tDP + cb, dpv);
-          tmem_wait_ld();
+          uint32_t dsk[16];
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
             const float4 Dl = d4[(cb >> 2) + c4];
-            const float dl[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
-            float ds[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              ds[e] = p[ch * 32 + 4 * c4 + e] * (__uint_as_float(dpv[4 * c4 + e]) - dl[e]);
-            dsk[2 * c4] = pack_bf16x2(ds[0], ds[1]);
-            dsk[2 * c4 + 1] = pack_bf16x2(ds[2], ds[3]);
+            const int e0 = ch * 32 + 4 * c4;
+            const float2 ds01 = fmul2(make_float2(p[e0], p[e0 + 1]),
+                                      fsub2(make_float2(__uint_as_float(dpv[e0]), __uint_as_float(dpv[e0 + 1])),
+                                            make_float2(Dl.x, Dl.y)));
+            const float2 ds23 = fmul2(make_float2(p[e0 + 2], p[e0 + 3]),
+                                      fsub2(make_float2(__uint_as_float(dpv[e0 + 2]), __uint_as_float(dpv[e0 + 3])),
+                                            make_float2(Dl.z, Dl.w)));
+            dsk[2 * c4] = pack_bf16x2(ds01.x, ds01.y);
+            dsk[2 * c4 + 1] = pack_bf16x2(ds23.x, ds23.y);
           }
           tmem_st16<0>(tDP + packed_col(cb), dsk);
         }
@@ -250,7 +294,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(acc_free);
     }
   } else {
-    regs_dec<88>();
+    regs_dec<104>();
   }
   if (warp == 8) {
     // ----------------------------------------------------------------- TMA --
@@ -315,53 +359,71 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 9) {
     // ----------------------------------------------------------------- MMA --
-    // One thread issues every MMA (the other lanes wait at the end).  The
-    // tensor pipe queues very few MMAs ahead of it, so a barrier wait between
-    // two MMA groups leaves the pipe idle; the wait for the next q tile's
-    // operands is therefore tested (Probe) between the MMAs of dV.
+    // One thread issues every MMA (the other lanes wait at the end).
     if (lane == 0) {
       const uint32_t tS = tmem_base + C::kColS, tDP = tmem_base + C::kColDP;
       const uint32_t tDV = tmem_base + C::kColDV, tDK = tmem_base + C::kColDK;
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
       uint32_t items = 0, q_cnt = 0;
       bool ok = true;
-      Probe pr;
       auto q_addr = [&](uint32_t cnt) {
         return smem_u32(smem + C::kOffQ + (2 * (cnt % C::kStages)) * C::kTileBytes);
       };
-      // One descriptor per operand tile; k-steps are constant offsets from it.
-      const uint64_t dK0 = smem_desc_sw128(aK, 16, 1024), dV0 = smem_desc_sw128(aV, 16, 1024);
+      // One descriptor per operand tile per MMA group; k-steps are constant
+      // offsets from it.
+      const uint32_t aP = smem_u32(sP);
+      // The barriers of the next MMA group are tested between the MMAs of the
+      // current one (Probe), so that their latency overlaps queued tensor work.
+      Probe pa, pb;
+      auto mid = [&](int kk) {
+        if (kk == 1 || kk == 6) {
+          pa.test();
+          pb.test();
+        }
+      };
       // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
       auto issue_st = [&](uint32_t aQ) {
-        const uint64_t dq = smem_desc_sw128(aQ, 16, 1024);
+        const uint64_t dK0 = smem_desc_sw128(aK, 16, 1024), dq = smem_desc_sw128(aQ, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
           mma_ss(tS, desc_at(dK0, off), desc_at(dq, off), C::kIdescST, kk > 0 ? 1u : 0u);
+          mid(kk);
         }
       };
       auto issue_dpt = [&](uint32_t adO) {
-        const uint64_t ddo = smem_desc_sw128(adO, 16, 1024);
+        const uint64_t dV0 = smem_desc_sw128(aV, 16, 1024), ddo = smem_desc_sw128(adO, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
           mma_ss(tDP, desc_at(dV0, off), desc_at(ddo, off), C::kIdescST, kk > 0 ? 1u : 0u);
+          mid(kk);
         }
       };
-      // acc += (packed TMEM operand) x (B MN-major over d); tests the probe
-      // between k-steps
-      auto issue_acc = [&](uint32_t t_acc, uint32_t t_a, uint32_t aB, bool first) {
-        const uint64_t db = smem_desc_sw128(aB, C::kSubBytes, 1024);
+      // dV += P^T dO: A = P^T (shared memory, K-major over q), B = dO (MN-major over d)
+      auto issue_dv = [&](uint32_t adO, bool first) {
+        const uint64_t da = smem_desc_sw128(aP, 16, 1024);
+        const uint64_t db = smem_desc_sw128(adO, C::kSubBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(t_acc, t_a + packed_kstep(kk), desc_at(db, kk * 2048), C::kIdescAcc,
-                 (first && kk == 0) ? 0u : 1u);
-          if (kk == 2 || kk == 6) pr.test();
+          mma_ss(tDV, desc_at(da, (kk >> 2) * C::kSubBytes + (kk & 3) * 32), desc_at(db, kk * 2048),
+                 C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+          mid(kk);
         }
       };
-      // Per q tile t the order is dV(t), S^T(t+1), dK(t), dP^T(t+1): dV(t) and
-      // S^T(t+1) run under the dS phase of t, dK(t) and dP^T(t+1) under the
-      // exponential phase of t+1.
+      // dK += dS^T Q: A = dS^T (packed bf16 in TMEM), B = Q (MN-major over d)
+      auto issue_dk = [&](uint32_t aQ, bool first) {
+        const uint64_t db = smem_desc_sw128(aQ, C::kSubBytes, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDK, tDP + packed_kstep(kk), desc_at(db, kk * 2048), C::kIdescAcc,
+                 (first && kk == 0) ? 0u : 1u);
+      };
+      auto q_full_of = [&](uint32_t cnt) { return &q_full[cnt % C::kStages]; };
+      auto q_phase_of = [&](uint32_t cnt) { return (cnt / C::kStages) & 1; };
+      // Per q tile t the order is S^T(t+1), dV(t), dK(t), dP^T(t+1): S^T(t+1)
+      // is issued as soon as the elementwise warps have read S^T(t) out of
+      // TMEM, so it runs under their exponential phase of t.
       for (int round = 0; ok; ++round) {
         const int w = snake_item(round, cta, grid);
         if (w >= P.n_items) break;
@@ -374,35 +436,50 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t base = q_cnt;
         q_cnt += n;
         if (!mbar_wait(kv_full, items & 1, abort_flag, P.err) ||
-            !mbar_wait(&q_full[base % C::kStages], (base / C::kStages) & 1, abort_flag, P.err))
+            !mbar_wait(q_full_of(base), q_phase_of(base), abort_flag, P.err))
           break;
         tc_fence_after();
         issue_st(q_addr(base));
         tc_commit(s_ready);
+        if (n > 1) {
+          pa.set(s_free, base & 1);
+          pb.set(q_full_of(base + 1), q_phase_of(base + 1));
+        }
         issue_dpt(q_addr(base) + C::kTileBytes);
         tc_commit(dp_ready);
         for (int t = 0; t < n; ++t) {
           const uint32_t cnt = base + t;
           const uint32_t aQ = q_addr(cnt), adO = aQ + C::kTileBytes;
-          if (!mbar_wait(pa_ready, cnt & 1, abort_flag, P.err) ||
+          if (t + 1 < n) {
+            if (!pa.finish(abort_flag, P.err) || !pb.finish(abort_flag, P.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            pa.set(pa_ready, cnt & 1);
+            issue_st(q_addr(cnt + 1));
+            tc_commit(s_ready);
+          } else {
+            pa.set(pa_ready, cnt & 1);
+          }
+          if (!pa.finish(abort_flag, P.err) ||
               (t == 0 && items > 0 && !mbar_wait(acc_free, (items - 1) & 1, abort_flag, P.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (t + 1 < n) pr.set(&q_full[(cnt + 1) % C::kStages], ((cnt + 1) / C::kStages) & 1);
-          issue_acc(tDV, tS, adO, t == 0);  // dV += P^T dO
-          if (t + 1 < n) {
-            if (!pr.finish(abort_flag, P.err)) { ok = false; break; }
-            tc_fence_after();
-            issue_st(q_addr(cnt + 1));
-            tc_commit(s_ready);
-          }
-          if (!mbar_wait(pb_ready, cnt & 1, abort_flag, P.err)) { ok = false; break; }
+          pa.set(pb_ready, cnt & 1);
+          issue_dv(adO, t == 0);
+          tc_commit(p_free);
+          if (!pa.finish(abort_flag, P.err)) { ok = false; break; }
           tc_fence_after();
-          issue_acc(tDK, tDP, aQ, t == 0);  // dK += dS^T Q
+          issue_dk(aQ, t == 0);
           tc_commit(&q_empty[cnt % C::kStages]);
           if (t + 1 < n) {
+            if (t + 2 < n) {
+              pa.set(s_free, (cnt + 1) & 1);
+              pb.set(q_full_of(cnt + 2), q_phase_of(cnt + 2));
+            }
             issue_dpt(q_addr(cnt + 1) + C::kTileBytes);
             tc_commit(dp_ready);
           }

@@ -285,13 +285,13 @@ __global__ void __launch_bounds__(384, 1)
         // max operations would put its full latency on every tile)
         float mp[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mp[i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 8; ++i) mp[i] = fmaxf(__uint_as_float(r[i]), __uint_as_float(r[8 + i]));
 #pragma unroll
-        for (int c = 8; c < 128; c += 8)
+        for (int c = 16; c < 128; c += 16)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) mp[i] = fmaxf(mp[i], __uint_as_float(r[c + i]));
-        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+          for (int i = 0; i < 8; ++i)
+            mp[i] = fmax3(mp[i], __uint_as_float(r[c + i]), __uint_as_float(r[c + 8 + i]));
+        const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
         const float m_tile = mx * sl2;
         float m_new = m;
         if (m_tile > m + kThresh || m == -INFINITY) m_new = fmaxf(m, m_tile);
@@ -303,27 +303,30 @@ __global__ void __launch_bounds__(384, 1)
         if (j > 0 && __any_sync(0xffffffffu, grow)) rescale_rows<D>(tO, f);
         m = m_new;
         const float base = ((m == -INFINITY) ? 0.f : m) - kPOff;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // row sum as 4 independent chains
+        // exponentials and row sum on packed pairs (the row sum as 4 chains)
+        const float2 sl = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+        float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         if constexpr (F8) {
 #pragma unroll
           for (int c = 0; c < 128; c += 4) {
-            const float x0 = fmaf(__uint_as_float(r[c]), sl2, -base);
-            const float x1 = fmaf(__uint_as_float(r[c + 1]), sl2, -base);
-            const float x2 = fmaf(__uint_as_float(r[c + 2]), sl2, -base);
-            const float x3 = fmaf(__uint_as_float(r[c + 3]), sl2, -base);
-            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-            ls[(c >> 2) & 3] += (p0 + p1) + (p2 + p3);
-            r[c >> 2] = pack_e4m3x4(p0, p1, p2, p3);  // r[c/4] was read at or before this step
+            const float2 x01 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl, nb);
+            const float2 x23 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl, nb);
+            const float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
+            const float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
+            ls2[0] = fadd2(ls2[0], p01);
+            ls2[1] = fadd2(ls2[1], p23);
+            r[c >> 2] = pack_e4m3x4(p01.x, p01.y, p23.x, p23.y);  // r[c/4] was read at or before this step
           }
         } else {
 #pragma unroll
           for (int c = 0; c < 128; c += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(r[c]), sl2, -base));
-            const float p1 = ex2(fmaf(__uint_as_float(r[c + 1]), sl2, -base));
-            ls[(c >> 1) & 3] += p0 + p1;
-            r[c >> 1] = pack_bf16x2(p0, p1);  // r[c/2] was read at or before this step
+            const float2 x = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl, nb);
+            const float2 p = make_float2(ex2(x.x), ex2(x.y));
+            ls2[(c >> 1) & 1] = fadd2(ls2[(c >> 1) & 1], p);
+            r[c >> 1] = pack_bf16x2(p.x, p.y);  // r[c/2] was read at or before this step
           }
         }
+        const float ls[4] = {ls2[0].x, ls2[0].y, ls2[1].x, ls2[1].y};
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tmem_st32<0>(tS + 0, r);
         if constexpr (!F8) tmem_st32<32>(tS + 32, r);
