@@ -17,8 +17,10 @@
 //      on rank owner + t): S^T = K Q^T, dP^T = V dO^T (TMEM), P^T (bf16, to
 //      shared memory) and dS^T (bf16, back into TMEM), dV += P^T dO,
 //      dK += dS^T Q (A from TMEM).
-//   3. dQ kernel (tc_dq.cu): one Q tile per work item, dQ accumulated in TMEM
-//      and written once; no reductions.
+//   3. dQ kernel: one Q tile per work item, dQ accumulated in TMEM and written
+//      once; no reductions.  At D = 128 with an even number of tiles per chunk
+//      it runs on two SMs per pair of Q tiles (tc_dq2.cu, cta_group::2 MMAs),
+//      otherwise on one SM per Q tile (tc_dq.cu).
 // Computing dQ in its own kernel recomputes S and dP once more but removes the
 // fp32 dQ reduction traffic, which on this GPU costs more than the extra
 // tensor work.
@@ -54,6 +56,9 @@ namespace bwd {
 template <int D>
 int launch_tc_dq(const BwdParams& P, const CUtensorMap& mq, const CUtensorMap& mk,
                  const CUtensorMap& mv, const CUtensorMap& mdo, int grid, cudaStream_t stream);
+// two-SM dQ kernel (tc_dq2.cu): D = 128 and an even number of tiles per chunk
+bool tc_dq2_supported(const BwdParams& P, int D);
+int launch_tc_dq2(const BwdParams& P, const void* k, const void* v, long rows, cudaStream_t stream);
 
 namespace {
 
@@ -582,7 +587,11 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
   tc_dkdv_kernel<D><<<grid, 384, DkdvCfg<D>::kSmemBytes, stream>>>(mq, mk, mv, mdo, P);
   prof_end(kKTcDkdv, stream);
   if (cudaGetLastError() != cudaSuccess) return -1;
-  if (launch_tc_dq<D>(P, mq, mk, mv, mdo, grid, stream) < 0) return -1;
+  if (tc_dq2_supported(P, D)) {
+    if (launch_tc_dq2(P, k, v, rows, stream) < 0) return -1;
+  } else if (launch_tc_dq<D>(P, mq, mk, mv, mdo, grid, stream) < 0) {
+    return -1;
+  }
   return 3;
 }
 
