@@ -338,8 +338,9 @@ const char* cpattn_status_str(int status);
  * cpattn_launch_count: number of kernels this library has enqueued so far in
  *   this process (all devices).
  * cpattn_set_path: 0 = automatic (tcgen05 kernels where the shape allows),
- *   1 = force the CUDA-core kernels.  Returns the previous setting.  For tests
- *   that compare the two kernel families.
+ *   1 = force the CUDA-core kernels, 2 = tcgen05 kernels on one SM each (the
+ *   two-SM dQ kernel off); any other value means 0.  Returns the previous
+ *   setting.  For tests that compare the kernel families.
  * cpattn_last_path: kernel family used by the last fwd/bwd call
  *   (0 tcgen05, 1 CUDA cores).
  * cpattn_debug_stall: n > 0 makes the next n tcgen05 forward launches omit one

@@ -97,12 +97,13 @@ int check_attention_shape(int B, int H, int S, int D, int cp_size, int causal, f
 void add_launches(int n) { g_launches += n; }
 
 unsigned* device_error_word() { return err_word(); }
+int kernel_path() { return g_path.load(); }
 }  // namespace cpattn
 
 namespace {
 
-bool use_tc_fwd(const AttnShape& sh) { return g_path.load() == 0 && tc_fwd_supported(sh); }
-bool use_tc_bwd(const AttnShape& sh) { return g_path.load() == 0 && tc_bwd_supported(sh); }
+bool use_tc_fwd(const AttnShape& sh) { return g_path.load() != 1 && tc_fwd_supported(sh); }
+bool use_tc_bwd(const AttnShape& sh) { return g_path.load() != 1 && tc_bwd_supported(sh); }
 
 }  // namespace
 
@@ -123,7 +124,7 @@ const char* cpattn_status_str(int s) {
 }
 
 long long cpattn_launch_count(void) { return g_launches.load(); }
-int cpattn_set_path(int path) { return g_path.exchange(path ? 1 : 0); }
+int cpattn_set_path(int path) { return g_path.exchange(path == 1 || path == 2 ? path : 0); }
 int cpattn_last_path(void) { return g_last_path.load(); }
 int cpattn_debug_stall(int n) { return g_stall.exchange(n < 0 ? 0 : n); }
 

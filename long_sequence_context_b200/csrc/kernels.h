@@ -64,6 +64,10 @@ int num_sms(int device);
 // once per device), or null when the lookup failed.
 unsigned* device_error_word();
 
+// Kernel family selected by cpattn_set_path: 0 automatic, 1 CUDA cores only,
+// 2 tcgen05 kernels on one SM each (no two-SM kernels).
+int kernel_path();
+
 // ---- tcgen05 GEMM (gemm.cu): C[M][N] = op(A) op(B) (+ bias[N]), bf16, fp32 accumulation.
 // a_mn: A stored [K][M] (else [M][K]); b_mn: B stored [K][N] (else [N][K]).
 // gemm_check: 0 when the sizes are supported (M, N, K >= 1, multiples of 8).

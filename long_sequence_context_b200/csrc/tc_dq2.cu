@@ -435,7 +435,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
 }  // namespace
 
-bool tc_dq2_supported(const BwdParams& P, int D) { return D == 128 && P.T % 2 == 0 && P.tiles % 2 == 0; }
+// (kernel path 2 keeps every tcgen05 kernel on one SM, for tests that compare)
+bool tc_dq2_supported(const BwdParams& P, int D) {
+  return kernel_path() != 2 && D == 128 && P.T % 2 == 0 && P.tiles % 2 == 0;
+}
 
 int launch_tc_dq2(const BwdParams& P, const void* k, const void* v, long rows, cudaStream_t stream) {
   using C = Dq2Cfg;

@@ -196,3 +196,39 @@ def test_any_chunk_length_fwd_bwd_vs_oracle(cp, B, H, S, D, cp_size, causal, dty
         cp.merge_(o_acc, l_acc, op, lp)
     assert cp.sync_status() == cp.OK
     assert_close(o_acc.cpu(), ro, dtype, "O from steps + merge")
+
+
+TWO_SM_CASES = [
+    (1, 2, 1024, 128, 2, True),    # 2 tiles per chunk: one pair per chunk
+    (1, 4, 4096, 128, 4, True),    # 4 tiles per chunk, 4 heads (head groups of 4)
+    (2, 2, 2048, 128, 2, False),
+]
+
+
+@pytest.mark.parametrize("B,H,S,D,cp_size,causal", TWO_SM_CASES)
+def test_two_sm_dq_matches_one_sm_dq(cp, B, H, S, D, cp_size, causal):
+    """The two-SM dQ kernel (a cluster of two CTAs per pair of Q tiles,
+    cta_group::2 MMAs) against the one-SM dQ kernel on the same inputs: the
+    same products in the same order per output row, so the fp32 sums, and
+    hence the bf16 dQ, can differ at most by the tensor core's internal
+    summation order -- one bf16 rounding step (2^-8 relative) of an element,
+    plus 2^-8 of the row's largest entry for sums near a rounding boundary of
+    a cancelling row.  dK and dV come from the same kernel on both paths."""
+    q, k, v, dout = make_qkv(B, H, S, D, torch.bfloat16, seed=400 + S + H)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = cp.fwd(qd, kd, vd, cp_size, causal)
+    dq2, dk2, dv2 = cp.bwd(qd, kd, vd, o, lse, dod, cp_size, causal)
+    prev = cp.set_path(2)
+    try:
+        dq1, dk1, dv1 = cp.bwd(qd, kd, vd, o, lse, dod, cp_size, causal)
+        assert cp.sync_status() == cp.OK
+        assert cp.last_path() == 0
+    finally:
+        cp.set_path(prev)
+    assert torch.equal(dk2, dk1) and torch.equal(dv2, dv1)
+    a, b = dq2.float(), dq1.float()
+    rowmax = b.abs().amax(dim=-1, keepdim=True)
+    bound = 2.0 ** -8 * (b.abs() + rowmax) + 1e-30
+    assert bool(((a - b).abs() <= bound).all()), float((a - b).abs().max())
+    rq, _, _ = orc.attn_bwd(np64(q), np64(k), np64(v), np64(dout), causal, D ** -0.5)
+    assert_close(dq2.cpu(), rq, torch.bfloat16, "dQ (two SMs)")
