@@ -142,3 +142,15 @@ def test_status_strings(cp):
 def test_set_path_roundtrip(cp):
     prev = cp.set_path(1)
     assert cp.set_path(prev) == 1
+
+
+def test_set_path_values(cp):
+    """0 automatic, 1 CUDA cores, 2 tcgen05 on one SM each; anything else is 0."""
+    prev = cp.set_path(2)
+    try:
+        assert cp.set_path(7) == 2
+        assert cp.set_path(1) == 0
+        assert cp.set_path(-3) == 1
+        assert cp.set_path(0) == 0
+    finally:
+        cp.set_path(prev)
