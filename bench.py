@@ -359,33 +359,6 @@ def time_workload(cp, w, dev, peaks, steps=5, warmup=3):
     return out
 
 
-def time_fwd_alone(cp, w, q, k, v, o, lse, peaks, steps=10, warmup=3):
-    """The headline workload's forward timed on its own (K forward calls back
-    to back on the resident inputs), beside its time inside the fwd + bwd step,
-    where the backward's power draw lowers the clocks."""
-    import torch
-    stream = torch.cuda.current_stream(q.device)
-    for _ in range(warmup):
-        cp.fwd(q, k, v, w.cp_size, w.causal, w.scale, out=o, lse=lse)
-    torch.cuda.synchronize(q.device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(q.device.index if q.device.index is not None else 0)
-    clocks.start()
-    e0.record(stream)
-    for _ in range(steps):
-        cp.fwd(q, k, v, w.cp_size, w.causal, w.scale, out=o, lse=lse)
-    e1.record(stream)
-    torch.cuda.synchronize(q.device)
-    clk = clocks.stop()
-    st = cp.sync_status()
-    if st != cp.OK:
-        raise RuntimeError(f"forward failed: {cp.status_str(st)}")
-    ms = e0.elapsed_time(e1) / steps
-    tfl = w.flops_fwd() / (ms * 1e-3) / 1e12
-    return {"ms": ms, "tflops": tfl, "frac_of_peak": tfl / peaks["bf16_tflops"], "steps": steps,
-            "l2": "inputs larger than L2; no flush", "clocks": clk}
-
-
 def time_fp8_fwd(cp, w, q, k, v, peaks, steps=10, warmup=3):
     """The e4m3 ring forward (cpattn_fwd_fp8) on the workload's inputs, already
     quantised (K/V kept in e4m3, as a context-parallel job would hold them),
@@ -599,10 +572,8 @@ def run_gpu(args, w):
 
     # ---- the other workloads and the standalone merge (device-timed, after the
     # headline region; each its own allocation) ----
-    per_config, merge, fp8, fwd_alone = None, None, None, None
+    per_config, merge, fp8 = None, None, None
     if not args.no_extra and world == 1:
-        if not args.fwd_only:
-            fwd_alone = time_fwd_alone(cp, w, qd, kd, vd, od, lsed, peaks, steps=args.steps)
         if w.D == 128 and w.dtype == "bf16":
             fp8 = time_fp8_fwd(cp, w, qd, kd, vd, peaks)
         per_config = {}
@@ -637,7 +608,6 @@ def run_gpu(args, w):
             "per_config": per_config,
             "merge": merge,
             "fp8_fwd": fp8,
-            "fwd_alone": fwd_alone,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
