@@ -259,6 +259,12 @@ def run_reference(args, w):
 MERGE_ROWS, MERGE_D = 1 << 20, 128
 
 
+def pre_bytes_per_row(D, elem=2):
+    """Backward preprocess: read a row of O and of dO and its LSE, write delta
+    and LSE * log2(e)."""
+    return 2 * D * elem + 4 + 2 * 4
+
+
 def merge_bytes_per_row(D):
     """Algorithmic bytes of one merged row: read O_acc, O_part (D fp32 each) and
     the two LSEs, write O_acc and LSE_acc."""
@@ -480,6 +486,17 @@ def run_gpu(args, w):
                 "frac": ach / peak, "frac_of_burst_peak": ach / peaks["bf16_tflops"],
                 "traffic": recorded_traffic(dom, w.name), "traffic_unit": "bytes per launch"}
 
+    # the backward preprocess (HBM-bound): O, dO read, LSE read, delta and
+    # LSE*log2(e) written, per row
+    pre_roof = None
+    if "bwd_delta" in per_kernel:
+        rows = w.B * w.H * w.S
+        by = rows * pre_bytes_per_row(w.D, 2 if w.dtype == "bf16" else 4)
+        gbs = by / (per_kernel["bwd_delta"]["ms_avg"] * 1e-3) / 1e9
+        pre_roof = {"bound": "hbm", "kernel": "bwd_delta", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "bytes_per_launch": by,
+                    "peak_kind": f"hbm_gbs ({peaks['source']})"}
+
     # ---- end to end through the public API with host buffers ----
     # Every step copies its inputs (q, k, v, dO) from pinned host memory and reads
     # its results (O, LSE, dQ, dK, dV) back.  Pipelined: device tensors are
@@ -605,6 +622,7 @@ def run_gpu(args, w):
             "peaks": peaks,
             "per_kernel_ms": per_kernel,
             "roofline": roof,
+            "preprocess_roofline": pre_roof,
             "per_config": per_config,
             "merge": merge,
             "fp8_fwd": fp8,

@@ -509,32 +509,54 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// delta_i = sum_d dO_id O_id and LSE_i * log2(e); one warp per row
+// delta_i = sum_d dO_id O_id and LSE_i * log2(e).  HBM-bound: each thread
+// reads 16-byte pieces of O and dO (D/8 threads per row), two rows per thread
+// so that four loads are in flight, and the row's partial sums meet through
+// shuffles among its D/8 lanes.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const float* __restrict__ lse,
                                                       float* __restrict__ delta,
                                                       float* __restrict__ lse2, long rows) {
-  const long row = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  constexpr int E = D / 32;  // elements per lane
-  float acc = 0.f;
-  const __nv_bfloat16* op = o + row * D + lane * E;
-  const __nv_bfloat16* dp = dout + row * D + lane * E;
+  constexpr int TPR = D / 8;                 // threads per row
+  constexpr int RPB = 256 / TPR;             // rows per pass of the block
+  const int sub = threadIdx.x % TPR, rl = threadIdx.x / TPR;
+  const long r0 = (long)blockIdx.x * (2 * RPB) + rl, r1 = r0 + RPB;
+  float acc[2] = {0.f, 0.f};
+  uint4 a[2], b[2];
 #pragma unroll
-  for (int e = 0; e < E; e += 2) {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(op + e);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(dp + e);
-    acc = fmaf(__low2float(a), __low2float(b), acc);
-    acc = fmaf(__high2float(a), __high2float(b), acc);
+  for (int k = 0; k < 2; ++k) {
+    const long row = k ? r1 : r0;
+    if (row < rows) {
+      a[k] = reinterpret_cast<const uint4*>(o + row * D)[sub];
+      b[k] = reinterpret_cast<const uint4*>(dout + row * D)[sub];
+    } else {
+      a[k] = b[k] = make_uint4(0, 0, 0, 0);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    delta[row] = acc;
-    lse2[row] = lse[row] * kLog2e;
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t ua[4] = {a[k].x, a[k].y, a[k].z, a[k].w}, ub[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&ua[e]);
+      const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&ub[e]);
+      acc[k] = fmaf(__low2float(x), __low2float(y), acc[k]);
+      acc[k] = fmaf(__high2float(x), __high2float(y), acc[k]);
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], off);
+  }
+  if (sub == 0) {
+    if (r0 < rows) {
+      delta[r0] = acc[0];
+      lse2[r0] = lse[r0] * kLog2e;
+    }
+    if (r1 < rows) {
+      delta[r1] = acc[1];
+      lse2[r1] = lse[r1] * kLog2e;
+    }
   }
 }
 
@@ -548,7 +570,8 @@ int launch_impl(const AttnShape& sh, const void* q, const void* k, const void* v
       !make_tmap_bf16_2d(&mv, v, rows, D, 64, 128) || !make_tmap_bf16_2d(&mdo, dout, rows, D, 64, 128))
     return -1;
   prof_begin(kKDelta, stream);
-  bwd_pre_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+  constexpr int kPreRows = 2 * 256 / (D / 8);  // rows per block of the preprocess
+  bwd_pre_kernel<D><<<(unsigned)((rows + kPreRows - 1) / kPreRows), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, ws_delta,
       ws_lse2, rows);
   prof_end(kKDelta, stream);

@@ -36,3 +36,9 @@ def test_merge_bytes_per_row():
     # read acc O + LSE, read part O + LSE, write acc O + LSE (fp32)
     assert bench.merge_bytes_per_row(128) == 1548
     assert bench.merge_bytes_per_row(64) == 3 * 64 * 4 + 12
+
+
+def test_pre_bytes_per_row():
+    # read O and dO rows (bf16) and LSE, write delta and LSE*log2(e)
+    assert bench.pre_bytes_per_row(128) == 2 * 128 * 2 + 12
+    assert bench.pre_bytes_per_row(64, 4) == 2 * 64 * 4 + 12
