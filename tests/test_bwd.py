@@ -202,6 +202,7 @@ TWO_SM_CASES = [
     (1, 2, 1024, 128, 2, True),    # 2 tiles per chunk: one pair per chunk
     (1, 4, 4096, 128, 4, True),    # 4 tiles per chunk, 4 heads (head groups of 4)
     (2, 2, 2048, 128, 2, False),
+    (1, 3, 1024, 128, 2, True),    # 3 heads: head groups of 1
 ]
 
 
