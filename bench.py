@@ -161,6 +161,23 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def e2e_chunks(w, want):
+    """Number of groups one end-to-end step is split into: a divisor of the
+    heads (B == 1) or of the batch, at most `want`."""
+    n = w.H if w.B == 1 else w.B
+    c = max(1, min(want, n))
+    while n % c:
+        c -= 1
+    return c
+
+
+def chunk_views(t, w, c):
+    """`c` contiguous views of a [B, H, S, ...] tensor: head groups when B == 1,
+    batch groups otherwise."""
+    dim = 1 if w.B == 1 else 0
+    return list(t.chunk(c, dim=dim))
+
+
 def max_over_ranks(x, world):
     """Largest value of x over all ranks (the job's time is its slowest rank)."""
     if world == 1:
@@ -573,30 +590,45 @@ def run_gpu(args, w):
 
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
+        # Each step is split into head groups (batch groups when B > 1), one
+        # public-API call per group, so that the first group's compute starts
+        # once its inputs are on the device and the last group's results leave
+        # while nothing else is pending: only 1/C of the first copy-in and of
+        # the last copy-out stay exposed.
+        n_chunks = e2e_chunks(w, args.e2e_chunks)
+        views = [(tuple(chunk_views(t, w, n_chunks) for t in d_in), tuple(chunk_views(t, w, n_chunks) for t in d_out),
+                  tuple(chunk_views(t, w, n_chunks) for t in h_out)) for d_in, d_out, h_out in sets]
+        h_in_v = tuple(chunk_views(t, w, n_chunks) for t in h_in)
+
         def run_pipelined(n):
             ev = lambda: torch.cuda.Event()
-            in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+            in_done = [[ev() for _ in range(n_chunks)] for _ in range(2)]
+            comp_done = [[ev() for _ in range(n_chunks)] for _ in range(2)]
+            out_done = [[ev() for _ in range(n_chunks)] for _ in range(2)]
             for i in range(n):
                 b = i % 2
-                d_in, d_out, h_out = sets[b]
+                d_in, d_out, h_out = views[b]
                 with torch.cuda.stream(s_in):
+                    for c in range(n_chunks):
+                        if i >= 2:
+                            s_in.wait_event(comp_done[b][c])   # step i-2 has read this group's inputs
+                        for h, d in zip(h_in_v, d_in):
+                            d[c].copy_(h[c], non_blocking=True)
+                        in_done[b][c].record(s_in)
+                for c in range(n_chunks):
+                    stream.wait_event(in_done[b][c])
                     if i >= 2:
-                        s_in.wait_event(comp_done[b])      # step i-2 has read this set's inputs
-                    for h, d in zip(h_in, d_in):
-                        d.copy_(h, non_blocking=True)
-                    in_done[b].record(s_in)
-                stream.wait_event(in_done[b])
-                if i >= 2:
-                    stream.wait_event(out_done[b])         # step i-2's results have left
-                compute(d_in, d_out)
-                comp_done[b].record(stream)
-                with torch.cuda.stream(s_out):
-                    s_out.wait_event(comp_done[b])
-                    for d, h in zip(d_out, h_out):
-                        h.copy_(d, non_blocking=True)
-                    out_done[b].record(s_out)
-            for e in out_done:
-                stream.wait_event(e)
+                        stream.wait_event(out_done[b][c])      # step i-2's results of this group have left
+                    compute(tuple(t[c] for t in d_in), tuple(t[c] for t in d_out))
+                    comp_done[b][c].record(stream)
+                    with torch.cuda.stream(s_out):
+                        s_out.wait_event(comp_done[b][c])
+                        for d, h in zip(d_out, h_out):
+                            h[c].copy_(d[c], non_blocking=True)
+                        out_done[b][c].record(s_out)
+            for row in out_done:
+                for e in row:
+                    stream.wait_event(e)
 
         def timed(fn, n):
             fn(1)
@@ -617,7 +649,9 @@ def run_gpu(args, w):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": pip_ms / n_e2e,
                "overlap": "double-buffered device tensors; H2D and D2H on two copy streams overlap the "
-                          "neighbouring steps' compute (first copy-in and last copy-out exposed)",
+                          "neighbouring steps' compute; each step runs as `chunks` head groups, so 1/chunks of "
+                          "the first copy-in and of the last copy-out stay exposed",
+               "chunks": n_chunks,
                "serial": {"value": job_tflops(f_fwd + f_bwd, n_e2e, ser_ms, world),
                           "ms_per_step": ser_ms / n_e2e}}
 
@@ -930,6 +964,8 @@ def main():
     ap.add_argument("--impl", default="cpattn", choices=["cpattn", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="head (or batch) groups per end-to-end step, overlapping the first copy-in and last copy-out")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fwd-only", action="store_true", help="time the forward alone (profiling)")
     ap.add_argument("--ring", action="store_true",

@@ -42,3 +42,31 @@ def test_pre_bytes_per_row():
     # read O and dO rows (bf16) and LSE, write delta and LSE*log2(e)
     assert bench.pre_bytes_per_row(128) == 2 * 128 * 2 + 12
     assert bench.pre_bytes_per_row(64, 4) == 2 * 64 * 4 + 12
+
+
+class _W:
+    def __init__(self, B, H):
+        self.B, self.H = B, H
+
+
+def test_e2e_chunks_divide_the_heads_or_batch():
+    assert bench.e2e_chunks(_W(1, 32), 4) == 4
+    assert bench.e2e_chunks(_W(1, 6), 4) == 3       # largest divisor of 6 not above 4
+    assert bench.e2e_chunks(_W(1, 2), 8) == 2
+    assert bench.e2e_chunks(_W(2, 32), 4) == 2      # batch groups when B > 1
+    assert bench.e2e_chunks(_W(1, 7), 1) == 1
+
+
+def test_chunk_views_are_contiguous_and_cover_the_tensor():
+    import torch
+    for B, H in ((1, 8), (2, 4)):
+        w = _W(B, H)
+        c = bench.e2e_chunks(w, 4)
+        for shape in ((B, H, 16, 8), (B, H, 16)):
+            t = torch.arange(torch.Size(shape).numel()).reshape(shape)
+            parts = bench.chunk_views(t, w, c)
+            assert len(parts) == c
+            assert all(p.is_contiguous() for p in parts)
+            assert torch.equal(torch.cat(parts, dim=1 if B == 1 else 0), t)
+            # views share the tensor's storage (copies into them land in place)
+            assert all(p.untyped_storage().data_ptr() == t.untyped_storage().data_ptr() for p in parts)
