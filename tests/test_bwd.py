@@ -233,3 +233,26 @@ def test_two_sm_dq_matches_one_sm_dq(cp, B, H, S, D, cp_size, causal):
     assert bool(((a - b).abs() <= bound).all()), float((a - b).abs().max())
     rq, _, _ = orc.attn_bwd(np64(q), np64(k), np64(v), np64(dout), causal, D ** -0.5)
     assert_close(dq2.cpu(), rq, torch.bfloat16, "dQ (two SMs)")
+
+
+@pytest.mark.parametrize("groups", [2, 4])
+def test_head_group_calls_match_one_call(cp, groups):
+    # Heads are independent problems: calling the forward and the backward on
+    # head-slice views (as the end-to-end benchmark does, to overlap its copies)
+    # gives every output bit for bit as one call on all heads.
+    B, H, S, D, cps = 1, 4, 2048, 128, 2
+    q, k, v, dout = make_qkv(B, H, S, D, torch.bfloat16, seed=321)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, dout))
+    o, lse = cp.fwd(qd, kd, vd, cps, True)
+    dq, dk, dv = cp.bwd(qd, kd, vd, o, lse, dod, cps, True)
+    og, lg = torch.full_like(o, float("nan")), torch.full_like(lse, float("nan"))
+    gq, gk, gv = (torch.full_like(t, float("nan")) for t in (dq, dk, dv))
+    ws = torch.empty(cp.bwd_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=qd.device)
+    for c in range(groups):
+        h = slice(c * H // groups, (c + 1) * H // groups)
+        cp.fwd(qd[:, h], kd[:, h], vd[:, h], cps, True, out=og[:, h], lse=lg[:, h])
+        cp.bwd(qd[:, h], kd[:, h], vd[:, h], og[:, h], lg[:, h], dod[:, h], cps, True, workspace=ws,
+               dq=gq[:, h], dk=gk[:, h], dv=gv[:, h])
+    assert cp.sync_status() == cp.OK
+    for name, a, b in (("O", o, og), ("LSE", lse, lg), ("dQ", dq, gq), ("dK", dk, gk), ("dV", dv, gv)):
+        assert torch.equal(a, b), name
